@@ -1,0 +1,59 @@
+"""Plant plausible mistakes in a copy of the oracle; some pin must catch each.
+
+The mutated copy is executed from source in a fresh module object; the real
+oracle module is never modified.
+"""
+
+import os
+import types
+
+import pytest
+
+import oracle_pins
+
+SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "oracle", "ref.py")
+
+MUTANTS = {
+    "sink term dropped from denominator": ("den += math.exp(float(sink) - m)", "den += 0.0"),
+    "sink exponent sign flipped": ("den += math.exp(float(sink) - m)", "den += math.exp(m - float(sink))"),
+    "sink left out of the running max": ("m = max(m, float(sink))", "m = m"),
+    "lse without the max": ("return e / den, m + math.log(den)", "return e / den, math.log(den)"),
+    "window one too wide": ("lo = max(0, i - window + 1)", "lo = max(0, i - window)"),
+    "window one too narrow": ("lo = max(0, i - window + 1)", "lo = max(0, i - window + 2)"),
+    "query excluded from its own window": ("return np.arange(lo, i + 1, dtype=np.int64)",
+                                           "return np.arange(lo, max(lo + 1, i), dtype=np.int64)"),
+    "rope sin sign": ("out[..., :half] = x1 * cos - x2 * sin", "out[..., :half] = x1 * cos + x2 * sin"),
+    "rope frequency exponent": ("-2.0 * k / rot_dims", "-1.0 * k / rot_dims"),
+    "rope interleaved partner": ("x2 = x[..., half:rot_dims]", "x2 = np.roll(x[..., :rot_dims], -1, axis=-1)[..., :half]"),
+    "scale ignored": ("return 1.0 / math.sqrt(d) if not scale else float(scale)", "return 1.0"),
+    "gqa map modulo": ("        g = h // group\n        keys = window_keys", "        g = h % Hkv\n        keys = window_keys"),
+    "scores against V": ("a = (K[keys] @ _f64(q_i)) * scale\n    s, lse", "a = (K[keys][:, :1] @ _f64(q_i)[:1]) * scale\n    s, lse"),
+    "ring slots off by one": ("return np.arange(min(L, capacity), dtype=np.int64)",
+                              "return np.arange(min(L, capacity) - 1, dtype=np.int64)"),
+    "sparse window misses newest": ("win = np.arange(max(0, L - recent), L, dtype=np.int64)",
+                                    "win = np.arange(max(0, L - recent - 1), L - 1, dtype=np.int64)"),
+    "combine counts sink per chunk": ("L += math.exp(float(sink) - M)", "L += len(parts) * math.exp(float(sink) - M)"),
+    "combine without rescale": ("o = sum(oc * math.exp(m - M) for m, _, oc in parts) / L",
+                                "o = sum(oc for m, _, oc in parts) / L"),
+}
+
+
+def _mutant(old, new):
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation anchor not unique or missing: {old!r}"
+    mod = types.ModuleType("oracle_mutant")
+    exec(compile(src.replace(old, new), "oracle_mutant", "exec"), mod.__dict__)
+    return mod
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name):
+    mod = _mutant(*MUTANTS[name])
+    failures = []
+    for check in oracle_pins.ALL_CHECKS:
+        try:
+            check(mod)
+        except Exception as e:  # AssertionError or a crash both count
+            failures.append(check.__name__)
+            break
+    assert failures, f"no pin caught mutant: {name}"
