@@ -1,0 +1,475 @@
+"""Benchmark of the attention-sink kernels on B200.
+
+Headline workload (one "step"): prefill of one MiMo SWA layer, batch 1,
+n = 32768, 64 Q / 8 KV heads, window 128, partial RoPE on 64 dims (theta 1e4),
+per-head sink; inputs synthetic N(0,1) bf16, resident in HBM and larger than L2.
+``value`` is algorithmic TFLOP/s (2 * (192 + 128) * scored pairs * Hq / time).
+The same JSON line also carries, under ``workloads``, the GA-layer prefill
+(n = 32768 causal, 64/4), one hybrid decode step over the 48-layer pattern
+(B = 64) and the token-level sparse decode (B = 8, L = 262144, 128 + 1024), each
+with its roofline.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+Under torchrun each rank runs its own copy of the workload (weak scaling); the
+job time is the max over ranks.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from hybrid_sliding_window_sink_b200 import dist as D  # noqa: E402
+from hybrid_sliding_window_sink_b200 import workloads as wl  # noqa: E402
+
+METRIC = "prefill attn TFLOP/s & decode HBM GB/s, % of B200 roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ----------------------------------------------------------------------------- peaks / clocks
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed loop runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.path = None
+        try:
+            uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+            fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", uuid, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.close()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax = float(parts[2])
+                except ValueError:
+                    continue
+                for nm, val in zip(names, parts[5:9]):
+                    if val.lower().startswith("active"):
+                        reasons.add(nm)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------- algorithmic work
+def swa_pairs(n, window):
+    if window <= 0 or window >= n:
+        return n * (n + 1) // 2
+    return n * window - window * (window - 1) // 2
+
+
+def prefill_work(case: wl.PrefillCase):
+    pairs = swa_pairs(case.seqlen, case.window) * case.batch
+    flops = 2.0 * (wl.DQK + wl.DV) * pairs * case.hq
+    n, B = case.seqlen, case.batch
+    bytes_ = (B * n * case.hq * wl.DQK * 2 + B * n * case.hkv * (wl.DQK + wl.DV) * 2
+              + B * n * case.hq * wl.DV * 2 + B * case.hq * n * 4 + case.hq * 4)
+    return flops, float(bytes_)
+
+
+def decode_layer_bytes(lengths, hq, hkv, kind, cap):
+    L = np.asarray(lengths, dtype=np.int64)
+    keys = np.minimum(L, cap) if kind == "ring" else L
+    kv = int(keys.sum()) * hkv * (wl.DQK + wl.DV) * 2
+    B = len(L)
+    return float(kv + B * hq * wl.DQK * 2 + B * hq * wl.DV * 2 + B * hq * 4 + hq * 4 + B * 4)
+
+
+# ----------------------------------------------------------------------------- timing
+def timed(fn, steps, warmup, stream, flush=None):
+    """Run ``warmup`` untimed steps, then time exactly ``steps`` with CUDA events on
+    ``stream``, bracketed by barrier + synchronize. Returns elapsed ms of this rank."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    D.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        if flush is not None:
+            flush()
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    D.barrier()
+    return e0.elapsed_time(e1)
+
+
+def roofline_hbm(bytes_per_launch, ms_per_launch, peaks, tag, traffic=None):
+    ach = bytes_per_launch / (ms_per_launch * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": round(ach / peaks["hbm_gbs"], 4), "traffic": traffic, "peak_source": tag}
+
+
+def roofline_tensor(flops_per_launch, ms_per_launch, peak, tag, traffic=None):
+    ach = flops_per_launch / (ms_per_launch * 1e-3) / 1e12
+    return {"bound": "tensor", "achieved": round(ach, 2), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(ach / peak, 4), "traffic": traffic, "peak_source": tag}
+
+
+# ----------------------------------------------------------------------------- CPU oracle baseline
+def oracle_swa_sample(case: wl.PrefillCase, positions: int):
+    """Times the float64 oracle, as it stands, on query positions 0..positions-1 (all
+    heads) of the SWA-layer workload; returns (TFLOP/s, description, threads, seconds)."""
+    from oracle import ref
+    from threadpoolctl import threadpool_limits
+    inp = wl.prefill_inputs(case.batch, positions, case.hq, case.hkv, seed=case.seed)
+    q = wl.to_f64(inp["q"])
+    k, v, s = wl.to_f64(inp["k"]), wl.to_f64(inp["v"]), wl.to_f64(inp["sink"])
+    with threadpool_limits(1):
+        t0 = time.perf_counter()
+        ref.prefill(q, k, v, s, case.window, case.theta, wl.ROT_DIMS)
+        dt = time.perf_counter() - t0
+    pairs = swa_pairs(positions, case.window)
+    flops = 2.0 * (wl.DQK + wl.DV) * pairs * case.hq * case.batch
+    desc = (f"float64 oracle, all {case.hq} heads of query positions 0..{positions - 1} of the "
+            f"n={case.seqlen} SWA layer (same window, RoPE and sinks), one thread")
+    return flops / dt / 1e12, desc, 1, dt
+
+
+def oracle_positions_for(case, seconds):
+    """Query positions whose oracle run takes about ``seconds`` on this host."""
+    _, _, _, dt = oracle_swa_sample(case, 64)
+    per_pos = dt / 64
+    return int(max(32, min(4096, seconds / per_pos)))
+
+
+# ----------------------------------------------------------------------------- workloads
+def bench_prefill(case, steps, warmup, peaks, tag, dev, stream):
+    from hybrid_sliding_window_sink_b200 import _lib
+    inp = wl.case_prefill_inputs(case, device=dev)
+    out = torch.empty(case.batch, case.seqlen, case.hq, wl.DV, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(case.batch, case.hq, case.seqlen, dtype=torch.float32, device=dev)
+
+    def step():
+        _lib.prefill(inp["q"], inp["k"], inp["v"], inp["sink"], window=case.window,
+                     rope_theta=case.theta, rot_dims=wl.ROT_DIMS, out=out, lse=lse, stream=stream)
+
+    ms = timed(step, steps, warmup, stream)
+    flops, bytes_ = prefill_work(case)
+    err = _lib.last_device_error()
+    res = {"inp": inp, "ms_total": ms, "flops": flops, "bytes": bytes_, "device_error": err}
+    return res
+
+
+def e2e_prefill(case, steps, dev, stream):
+    """Same metric through the public call with host buffers: pinned H2D of the step's
+    inputs, the kernel, D2H of the outputs, all inside the timed region."""
+    from hybrid_sliding_window_sink_b200 import _lib
+    host = wl.case_prefill_inputs(case, device="cpu")
+    host = {k: v.pin_memory() for k, v in host.items()}
+    dq = torch.empty_like(host["q"], device=dev)
+    dk = torch.empty_like(host["k"], device=dev)
+    dv = torch.empty_like(host["v"], device=dev)
+    ds = torch.empty_like(host["sink"], device=dev)
+    out = torch.empty(case.batch, case.seqlen, case.hq, wl.DV, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(case.batch, case.hq, case.seqlen, dtype=torch.float32, device=dev)
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+
+    def step():
+        with torch.cuda.stream(stream):
+            dq.copy_(host["q"], non_blocking=True)
+            dk.copy_(host["k"], non_blocking=True)
+            dv.copy_(host["v"], non_blocking=True)
+            ds.copy_(host["sink"], non_blocking=True)
+            _lib.prefill(dq, dk, dv, ds, window=case.window, rope_theta=case.theta,
+                         rot_dims=wl.ROT_DIMS, out=out, lse=lse, stream=stream)
+            h_out.copy_(out, non_blocking=True)
+            h_lse.copy_(lse, non_blocking=True)
+
+    ms = timed(step, steps, 1, stream)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = h_out.numel() * h_out.element_size() + h_lse.numel() * h_lse.element_size()
+    return ms / steps, h2d, d2h
+
+
+def bench_decode_step(steps, warmup, peaks, tag, dev, stream):
+    """One decode step over the 48-layer hybrid pattern (B=64): 39 SWA ring layers with
+    distinct caches and 9 GA layers reading one padded linear cache (131072 slots)."""
+    from hybrid_sliding_window_sink_b200 import _lib
+    cs, cg = wl.HYBRID_DECODE_SWA, wl.HYBRID_DECODE_GA
+    L = wl.lengths_uniform(cs.batch, cs.min_len, cs.max_len, seed=cs.seed)
+    Ld = L.to(dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(cs.seed)
+    pattern = wl.layer_pattern()
+    layers = []
+    ga_k = torch.randn(cg.batch, cg.capacity, cg.hkv, wl.DQK, generator=g, device=dev,
+                       dtype=torch.float32).to(torch.bfloat16)
+    ga_v = torch.randn(cg.batch, cg.capacity, cg.hkv, wl.DV, generator=g, device=dev,
+                       dtype=torch.float32).to(torch.bfloat16)
+    for li, kind in enumerate(pattern):
+        hkv = cs.hkv if kind == 1 else cg.hkv
+        q = torch.randn(cs.batch, cs.hq, wl.DQK, generator=g, device=dev).to(torch.bfloat16)
+        sink = torch.randn(cs.hq, generator=g, device=dev)
+        if kind == 1:
+            kc = torch.randn(cs.batch, cs.capacity, hkv, wl.DQK, generator=g, device=dev).to(torch.bfloat16)
+            vc = torch.randn(cs.batch, cs.capacity, hkv, wl.DV, generator=g, device=dev).to(torch.bfloat16)
+        else:
+            kc, vc = ga_k, ga_v
+        out = torch.empty(cs.batch, cs.hq, wl.DV, dtype=torch.bfloat16, device=dev)
+        lse = torch.empty(cs.batch, cs.hq, dtype=torch.float32, device=dev)
+        layers.append((kind, q, kc, vc, sink, out, lse))
+    nws = _lib.workspace_size(cg.batch, cg.hq, cg.hkv, op=_lib.MIMO_OP_DECODE,
+                              kind=_lib.MIMO_CACHE_LINEAR, capacity=cg.capacity)
+    ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
+
+    def run_layer(lay):
+        kind, q, kc, vc, sink, out, lse = lay
+        _lib.decode(q, kc, vc, Ld, sink, kind="ring" if kind == 1 else "linear",
+                    out=out, lse=lse, workspace=ws, stream=stream)
+
+    def step():
+        for lay in layers:
+            run_layer(lay)
+
+    ms = timed(step, steps, warmup, stream)
+    Ls = L.tolist()
+    b_swa = decode_layer_bytes(Ls, cs.hq, cs.hkv, "ring", cs.capacity)
+    b_ga = decode_layer_bytes(Ls, cg.hq, cg.hkv, "linear", cg.capacity)
+    total = 39 * b_swa + 9 * b_ga
+    # per-kind kernel time: time GA layers and SWA layers separately
+    ga_layers = [l for l in layers if l[0] == 0]
+    swa_layers = [l for l in layers if l[0] == 1]
+    ms_ga = timed(lambda: [run_layer(l) for l in ga_layers], steps, 1, stream) / (steps * 9)
+    ms_swa = timed(lambda: [run_layer(l) for l in swa_layers], steps, 1, stream) / (steps * 39)
+    res = {
+        "value": round(total / (ms / steps * 1e-3) / 1e9, 1), "unit": "GB/s",
+        "ms_per_step": round(ms / steps, 4), "bytes_per_step": total,
+        "launches_per_step": 39 + 9 * 2,
+        "ga_layer": roofline_hbm(b_ga, ms_ga, peaks, tag),
+        "swa_layer": roofline_hbm(b_swa, ms_swa, peaks, tag),
+        "roofline": roofline_hbm(total, ms / steps, peaks, tag),
+        "ms_ga_layer": round(ms_ga, 4), "ms_swa_layer": round(ms_swa, 5),
+        "cache": "39 distinct SWA ring caches; one padded GA cache [64,131072,4,*] read by all 9 GA layers",
+        "l2": "GA layers read 11 GB each (>> L2); SWA ring caches 44.6 MB each, distinct per layer",
+    }
+    del layers, ga_k, ga_v, ws
+    return res
+
+
+def bench_sparse(steps, warmup, peaks, tag, dev, stream, calls=16):
+    """Token-level sparse decode: ``calls`` independent calls (distinct q and index sets,
+    >= 385 MB of gathered rows in all, more than L2) per step, captured in a CUDA graph."""
+    from hybrid_sliding_window_sink_b200 import _lib
+    c = wl.SPARSE_DECODE
+    lengths = [c.context] * c.batch
+    base = wl.decode_inputs(c.batch, c.hq, c.hkv, c.context, lengths, seed=c.seed, device=dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(c.seed + 1)
+    sets = []
+    nws = _lib.workspace_size(c.batch, c.hq, c.hkv, op=_lib.MIMO_OP_SPARSE, capacity=c.context,
+                              recent=c.recent, n_sel=c.n_sel)
+    for i in range(calls):
+        q = torch.randn(c.batch, c.hq, wl.DQK, generator=g, device=dev).to(torch.bfloat16)
+        sel = wl.sorted_unique_indices(c.batch, c.hkv, c.n_sel, [c.context - c.recent] * c.batch,
+                                       seed=c.seed + 100 + i).to(dev)
+        out = torch.empty(c.batch, c.hq, wl.DV, dtype=torch.bfloat16, device=dev)
+        lse = torch.empty(c.batch, c.hq, dtype=torch.float32, device=dev)
+        ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
+        sets.append((q, sel, out, lse, ws))
+
+    def calls_fn():
+        for (q, sel, out, lse, ws) in sets:
+            _lib.sparse(q, base["k_cache"], base["v_cache"], base["lengths"], sel, base["sink"],
+                        recent=c.recent, out=out, lse=lse, workspace=ws, stream=stream)
+
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    calls_fn()   # loads the library and warms caches outside capture
+    torch.cuda.synchronize()
+    with torch.cuda.graph(graph, stream=stream):
+        calls_fn()
+    ms = timed(graph.replay, steps, warmup, stream)
+    per_call_bytes = (c.batch * c.hkv * (c.recent + c.n_sel) * (wl.DQK + wl.DV) * 2
+                      + c.batch * c.hkv * c.n_sel * 4 + c.batch * c.hq * (wl.DQK + wl.DV) * 2
+                      + c.batch * c.hq * 4 + c.hq * 4 + c.batch * 4)
+    ms_call = ms / (steps * calls)
+    res = {"value": round(per_call_bytes / (ms_call * 1e-3) / 1e9, 1), "unit": "GB/s",
+           "ms_per_call": round(ms_call, 5), "bytes_per_call": per_call_bytes, "calls_per_step": calls,
+           "launches_per_call": 2, "roofline": roofline_hbm(per_call_bytes, ms_call, peaks, tag),
+           "graph": True}
+    del graph, sets, base
+    return res
+
+
+# ----------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="mimo", choices=["mimo", "reference"])
+    ap.add_argument("--only-main", action="store_true", help="skip the extra workloads")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    args = ap.parse_args()
+    warmup = max(3, args.warmup)
+    case = wl.SWA_PREFILL
+    peaks, tag = load_peaks()
+
+    if args.impl == "reference":
+        world, rank, _ = D.env_world()
+        if rank != 0:
+            return
+        # size each step so that warm-up + steps take about two minutes in all
+        positions = oracle_positions_for(case, 120.0 / (args.steps + warmup))
+        for _ in range(warmup):
+            oracle_swa_sample(case, positions)
+        times, vals = [], []
+        for _ in range(args.steps):
+            v, desc, cores, dt = oracle_swa_sample(case, positions)
+            vals.append(v)
+            times.append(dt)
+        value = sum(v * t for v, t in zip(vals, times)) / sum(times)
+        line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": warmup,
+                "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": case.name, "global_batch": case.batch, "seq_len": case.seqlen,
+                           "parallelism": "none (host CPU)"},
+                "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores,
+                                 "kind": "oracle", "sample": desc},
+                "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    world, rank = D.init("nccl")
+    _, _, local = D.env_world()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    from hybrid_sliding_window_sink_b200 import _lib
+    _lib.lib()
+    stream = torch.cuda.current_stream(dev)
+
+    # ---- headline: SWA-layer prefill (each rank its own copy: weak scaling)
+    clocks = ClockSampler(local)
+    res = bench_prefill(case, args.steps, warmup, peaks, tag, dev, stream)
+    clk = clocks.stop()
+    ms_rank = res["ms_total"]
+    ms_max = D.max_over_ranks(ms_rank, device=dev)
+    ms_step = ms_max / args.steps
+    flops, bytes_ = res["flops"], res["bytes"]
+    value = world * flops / (ms_step * 1e-3) / 1e12
+    del res["inp"]
+    torch.cuda.empty_cache()
+
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": warmup, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic N(0,1) bf16 Q/K/V, fp32 N(0,1) sinks, seeded",
+        "config": {"workload": case.name, "global_batch": case.batch * world, "seq_len": case.seqlen,
+                   "parallelism": f"dp{world} (independent problems per rank)",
+                   "l2": "inputs larger than L2 (1.52 GB per step)"},
+        "roofline": roofline_hbm(bytes_, ms_step, peaks, tag),
+        "tensor": roofline_tensor(flops, ms_step, peaks["bf16_tflops"], tag),
+        "gpu_launches": args.steps,
+        "clocks": clk,
+        "device_error": res["device_error"],
+    }
+
+    # ---- end to end through the public call with host buffers
+    if args.e2e_steps > 0:
+        e2e_ms, h2d, d2h = e2e_prefill(case, args.e2e_steps, dev, stream)
+        e2e_ms = D.max_over_ranks(e2e_ms, device=dev)
+        line["e2e"] = {"value": round(world * flops / (e2e_ms * 1e-3) / 1e12, 4), "unit": "TFLOP/s",
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                       "ms_per_step": round(e2e_ms, 3)}
+        torch.cuda.empty_cache()
+
+    # ---- the other workloads (single GPU figures, rank 0 reports its own)
+    if not args.only_main:
+        wls = {}
+        ksteps = max(3, min(args.steps // 20, 10))
+        try:
+            ga = bench_prefill(wl.GA_PREFILL, ksteps, 3, peaks, tag, dev, stream)
+            ms_ga = ga["ms_total"] / ksteps
+            wls["ga_prefill"] = {
+                "workload": wl.GA_PREFILL.name, "value": round(ga["flops"] / (ms_ga * 1e-3) / 1e12, 2),
+                "unit": "TFLOP/s", "ms_per_step": round(ms_ga, 4),
+                "roofline": roofline_tensor(ga["flops"], ms_ga, peaks["bf16_tflops"], tag),
+                "device_error": ga["device_error"]}
+            del ga
+            torch.cuda.empty_cache()
+        except Exception as e:  # report, do not hide
+            wls["ga_prefill"] = {"error": repr(e)}
+        try:
+            wls["hybrid_decode_step"] = bench_decode_step(max(3, ksteps), 3, peaks, tag, dev, stream)
+            wls["hybrid_decode_step"]["workload"] = "hybrid decode step, 48 layers, B=64"
+            torch.cuda.empty_cache()
+        except Exception as e:
+            wls["hybrid_decode_step"] = {"error": repr(e)}
+        try:
+            wls["sparse_decode"] = bench_sparse(max(5, ksteps), 3, peaks, tag, dev, stream)
+            wls["sparse_decode"]["workload"] = wl.SPARSE_DECODE.name
+            torch.cuda.empty_cache()
+        except Exception as e:
+            wls["sparse_decode"] = {"error": repr(e)}
+        line["workloads"] = wls
+
+    # ---- CPU oracle baseline (rank 0, N = 1 only)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, desc, cores, dt = oracle_swa_sample(case, oracle_positions_for(case, 15.0))
+        line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                                "sample": desc, "seconds": round(dt, 2)}
+
+    if rank == 0:
+        print(json.dumps(line))
+    D.finalize()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,401 @@
+// mimo_attn.cu - the C ABI of libmimo_attn.so (declared in include/mimo_attn.h):
+// host-side argument checks, tensor-map encoding, kernel selection and launches.
+// One translation unit holds every kernel so that they share the device error word.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "mimo_attn.h"
+#include "ptx.cuh"
+#include "decode.cuh"
+#include "prefill.cuh"
+
+namespace mimo {
+__device__ unsigned g_device_error = 0;
+}
+
+namespace {
+
+using mimo::DecodeParams;
+using mimo::PrefillParams;
+
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sm_count[kMaxDevices];
+std::atomic<unsigned*> g_err_ptr[kMaxDevices];
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// Current device and its SM count (148 on B200 when no device can be queried).
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return -1;
+  }
+  return dev;
+}
+
+int sm_count_for(int dev) {
+  if (dev < 0 || dev >= kMaxDevices) return 148;
+  int v = g_sm_count[dev].load(std::memory_order_relaxed);
+  if (v > 0) return v;
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    return 148;
+  }
+  g_sm_count[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
+
+unsigned* device_error_ptr(int dev) {
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
+  unsigned* p = g_err_ptr[dev].load(std::memory_order_acquire);
+  if (p) return p;
+  void* addr = nullptr;
+  if (cudaGetSymbolAddress(&addr, mimo::g_device_error) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  g_err_ptr[dev].store(static_cast<unsigned*>(addr), std::memory_order_release);
+  return static_cast<unsigned*>(addr);
+}
+
+bool group_ok(int g) { return g == 1 || g == 2 || g == 4 || g == 8 || g == 16; }
+
+mimo_status check_heads(const mimo_shape* s) {
+  if (!s) return MIMO_ERR_NULL;
+  if (s->batch < 1 || s->n_q_heads < 1 || s->n_kv_heads < 1) return MIMO_ERR_SHAPE;
+  if (s->n_q_heads % s->n_kv_heads) return MIMO_ERR_SHAPE;
+  if (!(s->softmax_scale == s->softmax_scale) || std::isinf(s->softmax_scale)) return MIMO_ERR_SHAPE;
+  if (s->head_dim_qk != mimo::kDQK || s->head_dim_v != mimo::kDV) return MIMO_ERR_UNSUPPORTED;
+  if (!group_ok(s->n_q_heads / s->n_kv_heads)) return MIMO_ERR_UNSUPPORTED;
+  if (s->batch > 65535) return MIMO_ERR_UNSUPPORTED;
+  return MIMO_OK;
+}
+
+float scale_log2_of(const mimo_shape* s) {
+  const float sc = s->softmax_scale > 0.f ? s->softmax_scale : 1.0f / std::sqrt(static_cast<float>(s->head_dim_qk));
+  return sc * 1.4426950408889634f;
+}
+
+// ---------------------------------------------------------------- tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    else
+      cudaGetLastError();
+  });
+  return fn;
+}
+
+// 4-D bf16 tensor [d3][d2][d1][d0] (d0 innermost), box {64, b1, b2, 1}, 128-byte swizzle.
+bool make_tmap(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t d3,
+               uint32_t b1, uint32_t b2) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[4] = {d0, d1, d2, d3};
+  cuuint64_t strides[3] = {d0 * 2, d0 * d1 * 2, d0 * d1 * d2 * 2};
+  cuuint32_t box[4] = {64, b1, b2, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------- prefill
+template <int G, int BN, int NKS>
+mimo_status launch_prefill(const mimo_shape* s, const void* q, const void* k, const void* v,
+                           PrefillParams prm, int sms, cudaStream_t st) {
+  using C = mimo::PfCfg<G, BN, NKS>;
+  CUtensorMap tq, tk, tv;
+  const uint64_t n = static_cast<uint64_t>(s->seqlen), B = static_cast<uint64_t>(s->batch);
+  if (!make_tmap(&tq, q, mimo::kDQK, s->n_q_heads, n, B, G, C::P) ||
+      !make_tmap(&tk, k, mimo::kDQK, s->n_kv_heads, n, B, 1, BN) ||
+      !make_tmap(&tv, v, mimo::kDV, s->n_kv_heads, n, B, 1, BN))
+    return MIMO_ERR_CUDA;
+  auto kern = mimo::prefill_kernel<G, BN, NKS>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess) {
+    cudaGetLastError();
+    return MIMO_ERR_CUDA;
+  }
+  prm.n_qtiles = (s->seqlen + C::P - 1) / C::P;
+  const long long work = static_cast<long long>(s->batch) * s->n_kv_heads * prm.n_qtiles;
+  if (work > 0x7fffffffLL) return MIMO_ERR_UNSUPPORTED;
+  prm.num_work = static_cast<int>(work);
+  const int grid = prm.num_work < sms ? prm.num_work : sms;
+  kern<<<grid, mimo::kPfThreads, C::SMEM, st>>>(tq, tk, tv, prm);
+  return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ERR_CUDA;
+}
+
+template <int G>
+mimo_status prefill_group(const mimo_shape* s, const void* q, const void* k, const void* v,
+                          const PrefillParams& prm, int sms, cudaStream_t st) {
+  constexpr int P = 128 / G;
+  const bool swa = prm.window > 0 && prm.window < s->seqlen;
+  // one 144-key tile covers the whole window of a row block when P + W - 1 <= 144
+  if (swa && P + prm.window - 1 <= 144) return launch_prefill<G, 144, 1>(s, q, k, v, prm, sms, st);
+  return launch_prefill<G, 128, 2>(s, q, k, v, prm, sms, st);
+}
+
+// ---------------------------------------------------------------- decode
+struct DecodePlan {
+  int chunk, nchunks, direct;
+  size_t bytes;
+};
+
+int pow2_floor(long long x) {
+  int r = 1;
+  while (static_cast<long long>(r) * 2 <= x && r < (1 << 30)) r *= 2;
+  return r;
+}
+
+DecodePlan plan_decode(const mimo_shape* s, int mode, int cap, int recent, int n_sel, int sms) {
+  DecodePlan pl{};
+  const long long units = static_cast<long long>(s->batch) * s->n_kv_heads;
+  long long total = mode == mimo::kModeSparse ? static_cast<long long>(recent) + n_sel : cap;
+  if (total < 1) total = 1;
+  if (mode == mimo::kModeSparse) {
+    // about one wave of two CTAs per SM
+    long long c = (total * units + 2LL * sms - 1) / (2LL * sms);
+    int ch = pow2_floor(c);
+    if (ch < c) ch *= 2;
+    pl.chunk = ch < 64 ? 64 : (ch > mimo::kDecMaxTokList ? mimo::kDecMaxTokList : ch);
+  } else if (total <= 256) {
+    pl.chunk = static_cast<int>((total + 63) / 64 * 64);
+  } else {
+    // several waves so that uneven lengths balance
+    const long long c = total * units / (16LL * sms);
+    const int ch = pow2_floor(c);
+    pl.chunk = ch < 256 ? 256 : (ch > 4096 ? 4096 : ch);
+  }
+  pl.nchunks = static_cast<int>((total + pl.chunk - 1) / pl.chunk);
+  pl.direct = pl.nchunks == 1;
+  if (pl.direct) {
+    pl.bytes = 0;
+  } else {
+    const size_t rows = static_cast<size_t>(s->batch) * s->n_q_heads * pl.nchunks;
+    const size_t ml = (rows * 2 * sizeof(float) + 255) / 256 * 256;
+    pl.bytes = ml + rows * mimo::kDV * sizeof(float);
+  }
+  return pl;
+}
+
+template <int G>
+mimo_status launch_decode_g(DecodeParams prm, cudaStream_t st) {
+  auto kern = mimo::decode_split_kernel<G>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, mimo::kDecSmemBytes) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return MIMO_ERR_CUDA;
+  }
+  dim3 grid(prm.nchunks, prm.Hkv, prm.B);
+  kern<<<grid, mimo::kDecThreads, mimo::kDecSmemBytes, st>>>(prm);
+  if (cudaGetLastError() != cudaSuccess) return MIMO_ERR_CUDA;
+  if (!prm.direct) {
+    mimo::decode_combine_kernel<<<prm.B * prm.Hq, mimo::kDV, 0, st>>>(prm);
+    if (cudaGetLastError() != cudaSuccess) return MIMO_ERR_CUDA;
+  }
+  return MIMO_OK;
+}
+
+mimo_status run_decode(const mimo_shape* s, int mode, const void* q, const void* kc, const void* vc,
+                       int cap, long long stride, const int* lengths, int recent, const int* sel,
+                       int n_sel, const float* sink, void* out, float* lse, void* ws, size_t ws_bytes,
+                       void* stream) {
+  mimo_status e = check_heads(s);
+  if (e != MIMO_OK) return e;
+  if (!q || !kc || !vc || !lengths || !out) return MIMO_ERR_NULL;
+  if (mode == mimo::kModeSparse && n_sel > 0 && !sel) return MIMO_ERR_NULL;
+  if (cap < 1 || stride < cap) return MIMO_ERR_SHAPE;
+  if (mode == mimo::kModeSparse && (recent < 0 || n_sel < 0)) return MIMO_ERR_SHAPE;
+  if (!aligned(q, 16) || !aligned(kc, 16) || !aligned(vc, 16) || !aligned(out, 16) ||
+      !aligned(lengths, 4) || (sel && !aligned(sel, 4)) || (sink && !aligned(sink, 4)) ||
+      (lse && !aligned(lse, 4)))
+    return MIMO_ERR_ALIGN;
+  const int dev = current_device();
+  if (dev < 0) return MIMO_ERR_CUDA;
+  const int sms = sm_count_for(dev);
+  const DecodePlan pl = plan_decode(s, mode, cap, recent, n_sel, sms);
+  if (pl.bytes > 0 && (!ws || ws_bytes < pl.bytes)) return MIMO_ERR_WORKSPACE;
+  if (ws && !aligned(ws, 16)) return MIMO_ERR_ALIGN;
+  DecodeParams prm{};
+  prm.q = static_cast<const __nv_bfloat16*>(q);
+  prm.k = static_cast<const __nv_bfloat16*>(kc);
+  prm.v = static_cast<const __nv_bfloat16*>(vc);
+  prm.lengths = lengths;
+  prm.sel = sel;
+  prm.sink = sink;
+  prm.out = static_cast<__nv_bfloat16*>(out);
+  prm.lse = lse;
+  if (pl.bytes > 0) {
+    const size_t rows = static_cast<size_t>(s->batch) * s->n_q_heads * pl.nchunks;
+    const size_t ml = (rows * 2 * sizeof(float) + 255) / 256 * 256;
+    prm.part_ml = static_cast<float*>(ws);
+    prm.part_o = reinterpret_cast<float*>(static_cast<char*>(ws) + ml);
+  }
+  prm.seq_stride = stride;
+  prm.B = s->batch;
+  prm.Hq = s->n_q_heads;
+  prm.Hkv = s->n_kv_heads;
+  prm.group = s->n_q_heads / s->n_kv_heads;
+  prm.cap = cap;
+  prm.mode = mode;
+  prm.chunk = pl.chunk;
+  prm.nchunks = pl.nchunks;
+  prm.recent = recent;
+  prm.n_sel = n_sel;
+  prm.direct = pl.direct;
+  prm.scale_log2 = scale_log2_of(s);
+  prm.err = device_error_ptr(dev);
+  if (!prm.err) return MIMO_ERR_CUDA;
+  if (s->n_kv_heads > 65535) return MIMO_ERR_UNSUPPORTED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  switch (prm.group) {
+    case 1: return launch_decode_g<1>(prm, st);
+    case 2: return launch_decode_g<2>(prm, st);
+    case 4: return launch_decode_g<4>(prm, st);
+    case 8: return launch_decode_g<8>(prm, st);
+    default: return launch_decode_g<16>(prm, st);
+  }
+}
+
+}  // namespace
+
+// ============================================================== C ABI
+extern "C" {
+
+mimo_status mimo_attn_prefill(const mimo_shape* s, const void* q, const void* k, const void* v,
+                              const float* sink, int window, float rope_theta, int rot_dims,
+                              void* out, float* lse, void* stream) {
+  mimo_status e = check_heads(s);
+  if (e != MIMO_OK) return e;
+  if (!q || !k || !v || !out) return MIMO_ERR_NULL;
+  if (s->seqlen < 1) return MIMO_ERR_SHAPE;
+  if (rot_dims < 0 || rot_dims > mimo::kDQK) return MIMO_ERR_SHAPE;
+  if (rot_dims % 16) return MIMO_ERR_UNSUPPORTED;
+  if (rot_dims > 0 && !(rope_theta > 0.f && std::isfinite(rope_theta))) return MIMO_ERR_SHAPE;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+      (sink && !aligned(sink, 4)) || (lse && !aligned(lse, 4)))
+    return MIMO_ERR_ALIGN;
+  const int dev = current_device();
+  if (dev < 0) return MIMO_ERR_CUDA;
+  PrefillParams prm{};
+  prm.sink = sink;
+  prm.out = static_cast<__nv_bfloat16*>(out);
+  prm.lse = lse;
+  prm.B = s->batch;
+  prm.n = s->seqlen;
+  prm.Hq = s->n_q_heads;
+  prm.Hkv = s->n_kv_heads;
+  prm.window = window;
+  prm.rot_dims = rot_dims;
+  prm.rope_theta = static_cast<double>(rope_theta);
+  prm.scale_log2 = scale_log2_of(s);
+  prm.err = device_error_ptr(dev);
+  if (!prm.err) return MIMO_ERR_CUDA;
+  const int sms = sm_count_for(dev);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  switch (s->n_q_heads / s->n_kv_heads) {
+    case 1: return prefill_group<1>(s, q, k, v, prm, sms, st);
+    case 2: return prefill_group<2>(s, q, k, v, prm, sms, st);
+    case 4: return prefill_group<4>(s, q, k, v, prm, sms, st);
+    case 8: return prefill_group<8>(s, q, k, v, prm, sms, st);
+    default: return prefill_group<16>(s, q, k, v, prm, sms, st);
+  }
+}
+
+mimo_status mimo_attn_decode(const mimo_shape* s, const void* q, const void* k_cache,
+                             const void* v_cache, int cache_kind, int cache_capacity,
+                             long long seq_stride_tokens, const int* lengths, const float* sink,
+                             void* out, float* lse, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+  if (cache_kind != MIMO_CACHE_RING && cache_kind != MIMO_CACHE_LINEAR) return MIMO_ERR_SHAPE;
+  const int mode = cache_kind == MIMO_CACHE_RING ? mimo::kModeRing : mimo::kModeLinear;
+  return run_decode(s, mode, q, k_cache, v_cache, cache_capacity, seq_stride_tokens, lengths, 0,
+                    nullptr, 0, sink, out, lse, workspace, workspace_bytes, stream);
+}
+
+mimo_status mimo_attn_sparse(const mimo_shape* s, const void* q, const void* k_cache,
+                             const void* v_cache, int cache_capacity, long long seq_stride_tokens,
+                             const int* lengths, int recent, const int* sel_idx, int n_sel,
+                             const float* sink, void* out, float* lse, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  return run_decode(s, mimo::kModeSparse, q, k_cache, v_cache, cache_capacity, seq_stride_tokens,
+                    lengths, recent, sel_idx, n_sel, sink, out, lse, workspace, workspace_bytes,
+                    stream);
+}
+
+size_t mimo_attn_workspace_size(const mimo_shape* s, int op, int cache_kind, int cache_capacity,
+                                int recent, int n_sel) {
+  if (check_heads(s) != MIMO_OK || cache_capacity < 1) return 0;
+  int mode;
+  if (op == MIMO_OP_SPARSE) {
+    if (recent < 0 || n_sel < 0) return 0;
+    mode = mimo::kModeSparse;
+  } else if (op == MIMO_OP_DECODE) {
+    if (cache_kind == MIMO_CACHE_RING) mode = mimo::kModeRing;
+    else if (cache_kind == MIMO_CACHE_LINEAR) mode = mimo::kModeLinear;
+    else return 0;
+  } else {
+    return 0;
+  }
+  return plan_decode(s, mode, cache_capacity, recent, n_sel, sm_count_for(current_device())).bytes;
+}
+
+mimo_status mimo_attn_check_indices(const mimo_shape* s, const int* lengths, const int* sel_idx,
+                                    int n_sel, int recent, int cache_capacity,
+                                    unsigned int* d_violations, void* stream) {
+  if (!s) return MIMO_ERR_NULL;
+  if (s->batch < 1 || s->n_kv_heads < 1 || n_sel < 0 || recent < 0 || cache_capacity < 1)
+    return MIMO_ERR_SHAPE;
+  if (!lengths || !d_violations || (n_sel > 0 && !sel_idx)) return MIMO_ERR_NULL;
+  const int rows = s->batch * s->n_kv_heads;
+  mimo::check_indices_kernel<<<(rows + 127) / 128, 128, 0, static_cast<cudaStream_t>(stream)>>>(
+      lengths, sel_idx, s->batch, s->n_kv_heads, n_sel, recent, cache_capacity, d_violations);
+  return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ERR_CUDA;
+}
+
+unsigned int mimo_attn_last_device_error(void) {
+  unsigned v = 0;
+  if (cudaDeviceSynchronize() != cudaSuccess) {
+    cudaGetLastError();
+    return 0xFFFFFFFFu;
+  }
+  if (cudaMemcpyFromSymbol(&v, mimo::g_device_error, sizeof(v)) != cudaSuccess) {
+    cudaGetLastError();
+    return 0xFFFFFFFFu;
+  }
+  const unsigned zero = 0;
+  cudaMemcpyToSymbol(mimo::g_device_error, &zero, sizeof(zero));
+  return v;
+}
+
+const char* mimo_status_string(mimo_status st) {
+  switch (st) {
+    case MIMO_OK: return "ok";
+    case MIMO_ERR_NULL: return "a required pointer is NULL";
+    case MIMO_ERR_SHAPE: return "sizes inconsistent or out of range";
+    case MIMO_ERR_UNSUPPORTED: return "unsupported head dims, group size or rot_dims";
+    case MIMO_ERR_ALIGN: return "misaligned data pointer";
+    case MIMO_ERR_WORKSPACE: return "workspace missing or too small";
+    case MIMO_ERR_CUDA: return "CUDA error";
+    case MIMO_ERR_DEVICE: return "kernel reported an internal timeout";
+  }
+  return "unknown status";
+}
+
+int mimo_attn_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,179 @@
+/*
+ * mimo_attn.h - C ABI of libmimo_attn.so: attention-sink softmax attention for
+ * hybrid sliding-window (SWA) / global (GA) decoder layers on NVIDIA B200 (sm_100a).
+ *
+ * What is computed ("MiMo-V2-Flash: Hybrid Sliding Window Attention
+ * Architecture", §4.4 and §5 steps 2-5). For query i, query head h and its key
+ * set J_i:
+ *
+ *   a_ij = (q_i . k_j) * scale                           (§1.2, scale = 1/sqrt(192))
+ *   m_i  = max(sink_h, max_{j in J_i} a_ij)
+ *   s_ij = exp(a_ij - m_i) / (exp(sink_h - m_i) + sum_{j' in J_i} exp(a_ij' - m_i))
+ *   o_i  = sum_{j in J_i} s_ij v_j                        (the sink has no value vector)
+ *   lse_i = m_i + ln(exp(sink_h - m_i) + sum_j exp(a_ij - m_i))   (natural log, sink included)
+ *
+ * J_i is the causal window W(i) = [max(0, i-W+1), i] on SWA layers (§2.1, 0-based)
+ * or the causal prefix [0, i] on GA layers. A NULL sink means exp(sink) = 0.
+ *
+ * Conventions shared by every call:
+ *  - bf16 tensors are passed as pointers to raw bf16 bits (__nv_bfloat16), row-major,
+ *    contiguous in the layout stated per argument. fp32 tensors are float.
+ *  - Every data pointer is a DEVICE pointer on the current CUDA device and must be
+ *    16-byte aligned (MIMO_ERR_ALIGN otherwise). `stream` is a cudaStream_t
+ *    (NULL = legacy default stream).
+ *  - Ownership: the caller owns every buffer. The library never allocates, frees
+ *    or synchronises; all work is enqueued on `stream` and the call returns
+ *    immediately.
+ *  - Errors: arguments are checked on the host before any launch; on error nothing
+ *    is launched and a status other than MIMO_OK is returned. A failed launch maps
+ *    to MIMO_ERR_CUDA. Contents of device arrays (lengths, indices) are not checked
+ *    by the fast path; kernels clamp them so that no access leaves the caller's
+ *    buffers, and mimo_attn_check_indices reports violations.
+ *  - Supported head dims: head_dim_qk = 192, head_dim_v = 128. n_q_heads must be a
+ *    multiple of n_kv_heads with group n_q_heads / n_kv_heads in {1, 2, 4, 8, 16};
+ *    query head h reads KV head h / group (contiguous groups).
+ *  - Thread safety: calls may be made from several host threads; the only shared
+ *    mutable state is the device error word read by mimo_attn_last_device_error.
+ */
+#ifndef MIMO_ATTN_H
+#define MIMO_ATTN_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum mimo_status {
+  MIMO_OK = 0,
+  MIMO_ERR_NULL = 1,        /* a required pointer is NULL */
+  MIMO_ERR_SHAPE = 2,       /* sizes inconsistent or out of range */
+  MIMO_ERR_UNSUPPORTED = 3, /* well-formed but not implemented (head dims, group size, rot_dims) */
+  MIMO_ERR_ALIGN = 4,       /* a data pointer is not 16-byte aligned */
+  MIMO_ERR_WORKSPACE = 5,   /* workspace NULL or smaller than mimo_attn_workspace_size() */
+  MIMO_ERR_CUDA = 6,        /* a CUDA call failed (no device, launch failure, ...) */
+  MIMO_ERR_DEVICE = 7       /* a kernel reported an internal timeout (see mimo_attn_last_device_error) */
+} mimo_status;
+
+/* Problem sizes. softmax_scale <= 0 selects 1/sqrt(head_dim_qk). */
+typedef struct mimo_shape {
+  int batch;        /* B */
+  int seqlen;       /* n (prefill only; ignored by decode / sparse) */
+  int n_q_heads;    /* Hq */
+  int n_kv_heads;   /* Hkv */
+  int head_dim_qk;  /* 192 */
+  int head_dim_v;   /* 128 */
+  float softmax_scale;
+} mimo_shape;
+
+enum { MIMO_CACHE_RING = 0, MIMO_CACHE_LINEAR = 1 };
+enum { MIMO_OP_DECODE = 0, MIMO_OP_SPARSE = 1 };
+
+/*
+ * Prefill of one layer over whole sequences ("MiMo-V2-Flash ..." §5 steps 2-5;
+ * partial RoPE from "...MiMo-V2.6-Flash-MOPD混合SWA设计原理" §5).
+ *
+ *  q    [B, n, Hq, 192]  bf16, un-rotated
+ *  k    [B, n, Hkv, 192] bf16, un-rotated
+ *  v    [B, n, Hkv, 128] bf16
+ *  sink [Hq] fp32, or NULL (no sink term)
+ *  window     W > 0 and W < n: SWA with J_i = [max(0, i-W+1), i]; W <= 0 or W >= n: GA (causal prefix)
+ *  rope_theta RoPE base (1e4 for SWA, 1e7 for GA); must be > 0 when rot_dims > 0
+ *  rot_dims   number of leading QK dims rotated at positions 0..n-1 with the rotate-half
+ *             pairing (d, d + rot_dims/2) and inverse frequency theta^(-2k/rot_dims);
+ *             0 or a multiple of 16 up to 192 (64 = 0.334 * 192 on MiMo)
+ *  out  [B, n, Hq, 128] bf16 (written)
+ *  lse  [B, Hq, n] fp32 natural-log LSE including the sink (written), or NULL
+ *
+ * Runs the sm_100a tensor-core kernel (TMA-staged tiles, tcgen05 MMAs with TMEM
+ * accumulators). Tiles fully outside the window or the causal prefix are skipped.
+ */
+mimo_status mimo_attn_prefill(const mimo_shape* shape, const void* q, const void* k,
+                              const void* v, const float* sink, int window,
+                              float rope_theta, int rot_dims, void* out, float* lse,
+                              void* stream);
+
+/*
+ * One-token decode over a KV cache (SWA ring pool of O(W) slots, or GA linear pool;
+ * "...MiMo-V2.5..." dual-pool KV cache; math as above with i = L_b - 1).
+ *
+ *  q        [B, Hq, 192] bf16, already rotated at position L_b - 1
+ *  k_cache  [B, seq_stride_tokens, Hkv, 192] bf16, rotated K
+ *  v_cache  [B, seq_stride_tokens, Hkv, 128] bf16
+ *  cache_kind MIMO_CACHE_RING: token p of sequence b lives in slot p mod cache_capacity and
+ *             the query attends slots [0, min(L_b, cache_capacity)) (the last
+ *             cache_capacity tokens, i.e. the window when capacity = W);
+ *             MIMO_CACHE_LINEAR: slot t holds token t; the query attends [0, L_b)
+ *  cache_capacity     slots per sequence (>= 1, <= seq_stride_tokens)
+ *  seq_stride_tokens  distance between sequences in tokens
+ *  lengths  [B] int32 device: L_b >= 1 tokens so far including the query's own token
+ *           (linear: L_b <= cache_capacity; values are clamped to the cache)
+ *  sink     [Hq] fp32 or NULL
+ *  out      [B, Hq, 128] bf16 (written); lse [B, Hq] fp32 or NULL
+ *  workspace  device scratch of at least mimo_attn_workspace_size(shape, MIMO_OP_DECODE, cache_kind,
+ *             cache_capacity, 0, 0) bytes (may be NULL when that size is 0)
+ *
+ * Split-KV: partial (m, l, o) per chunk of keys without the sink, then one combine
+ * that adds the sink term once.
+ */
+mimo_status mimo_attn_decode(const mimo_shape* shape, const void* q, const void* k_cache,
+                             const void* v_cache, int cache_kind, int cache_capacity,
+                             long long seq_stride_tokens, const int* lengths,
+                             const float* sink, void* out, float* lse, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
+/*
+ * Token-level sparse decode ("小米MiMo-V3的核心架构HySparse2" §四.3): one merged sink
+ * softmax over the most recent `recent` tokens {L_b-recent, ..., L_b-1} plus `n_sel`
+ * selected tokens, read from one linear cache.
+ *
+ *  q, k_cache, v_cache, lengths, sink, out, lse: as in mimo_attn_decode (linear cache)
+ *  cache_capacity   slots per sequence; lengths and indices are clamped to it
+ *  recent           size of the forced recent window (128 on MiMo), >= 0
+ *  sel_idx [B, Hkv, n_sel] int32 device: per (sequence, KV head) sorted unique token
+ *          indices in [0, L_b - recent), shared by the group's query heads
+ *  n_sel            number of selected tokens (1024 on MiMo), >= 0
+ *  workspace        at least mimo_attn_workspace_size(shape, MIMO_OP_SPARSE, MIMO_CACHE_LINEAR,
+ *                   cache_capacity, recent, n_sel) bytes
+ *
+ * The index list drives a row gather; no dense mask is formed. Duplicates or indices
+ * inside the recent window are a precondition violation (counted by
+ * mimo_attn_check_indices), not an error of this call.
+ */
+mimo_status mimo_attn_sparse(const mimo_shape* shape, const void* q, const void* k_cache,
+                             const void* v_cache, int cache_capacity,
+                             long long seq_stride_tokens, const int* lengths, int recent,
+                             const int* sel_idx, int n_sel, const float* sink, void* out,
+                             float* lse, void* workspace, size_t workspace_bytes,
+                             void* stream);
+
+/* Bytes of device workspace mimo_attn_decode / mimo_attn_sparse need for these sizes
+ * on the current device (0 when none is needed). Returns 0 for invalid arguments. */
+size_t mimo_attn_workspace_size(const mimo_shape* shape, int op, int cache_kind,
+                                int cache_capacity, int recent, int n_sel);
+
+/* Debug check of sparse-decode preconditions, on `stream`: counts, into the device
+ * word *d_violations (which the caller zeroes first), every (b, g) row whose
+ * indices are not strictly increasing, fall outside [0, L_b - recent), or whose
+ * L_b is outside [1, cache_capacity]. Never traps. */
+mimo_status mimo_attn_check_indices(const mimo_shape* shape, const int* lengths,
+                                    const int* sel_idx, int n_sel, int recent,
+                                    int cache_capacity, unsigned int* d_violations,
+                                    void* stream);
+
+/* Synchronises the current device, then returns and clears the device error word
+ * that kernels set when a bounded wait gives up (0 = none). Host-blocking; for tests
+ * and debugging. */
+unsigned int mimo_attn_last_device_error(void);
+
+/* Static description of a status code. */
+const char* mimo_status_string(mimo_status status);
+
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+int mimo_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MIMO_ATTN_H */

@@ -49,6 +49,7 @@ __all__ = [
     "sink_softmax",
     "attend_row",
     "prefill",
+    "prefill_rows",
     "decode",
     "sparse_decode",
     "sparse_key_set",
@@ -151,9 +152,13 @@ def attend_row(q_i, K, V, keys, sink, scale):
     o_i = sum_j s_ij v_j (the sink carries no value vector, §4.2).
     """
     keys = np.asarray(keys, dtype=np.int64)
-    a = (K[keys] @ _f64(q_i)) * scale
+    if keys.size and keys[-1] - keys[0] + 1 == keys.size and np.all(np.diff(keys) == 1):
+        Kj, Vj = K[keys[0]:keys[-1] + 1], V[keys[0]:keys[-1] + 1]   # contiguous: a view
+    else:
+        Kj, Vj = K[keys], V[keys]
+    a = (Kj @ _f64(q_i)) * scale
     s, lse = sink_softmax(a, sink)
-    o = s @ V[keys]
+    o = s @ Vj
     return o, lse
 
 
@@ -205,11 +210,36 @@ def prefill(q, k, v, sink, window: int, rope_theta: float, rot_dims: int,
                     o[b, i, h], lse[b, h, i] = one(b, h, i, qr[b, i, h])
         return o, lse
     rows = list(rows)
+    q_rows = np.stack([q[b, i, h] for (b, h, i) in rows]) if rows else np.zeros((0, D))
+    return prefill_rows(q_rows, k, v, sink, window, rope_theta, rot_dims, rows, Hq, scale)
+
+
+def prefill_rows(q_rows, k, v, sink, window: int, rope_theta: float, rot_dims: int, rows,
+                 n_q_heads: int, scale: float | None = None):
+    """``prefill`` for selected rows only, without materialising all of Q.
+
+    q_rows[r] is the un-rotated query of rows[r] = (b, h, i); k, v are the full
+    [B, n, Hkv, D] tensors; query head h reads KV head h // (n_q_heads // Hkv).
+    Returns (o [len(rows), Dv], lse [len(rows)]).
+    """
+    k, v = _f64(k), _f64(v)
+    B, n, Hkv, D = k.shape
+    if n_q_heads % Hkv:
+        raise ValueError("Hq must be a multiple of Hkv")
+    group = n_q_heads // Hkv
+    sc = _scale(scale, D)
+    pos = np.arange(n, dtype=np.float64)
+    kr = np.stack([rope(k[b], pos, rope_theta, rot_dims) for b in range(B)])
+    sinks = None if sink is None else _f64(sink)
+    rows = list(rows)
     o = np.zeros((len(rows), v.shape[-1]))
     lse = np.zeros(len(rows))
     for r, (b, h, i) in enumerate(rows):
-        qrow = rope(q[b, i:i + 1, h:h + 1, :], pos[i:i + 1], rope_theta, rot_dims)[0, 0]
-        o[r], lse[r] = one(b, h, i, qrow)
+        g = h // group
+        qrow = rope(_f64(q_rows[r])[None, None, :], pos[i:i + 1], rope_theta, rot_dims)[0, 0]
+        keys = window_keys(i, window, n)
+        o[r], lse[r] = attend_row(qrow, kr[b, :, g, :], v[b, :, g, :], keys,
+                                  None if sinks is None else sinks[h], sc)
     return o, lse
 
 

@@ -155,6 +155,18 @@ def check_against_sdpa(ref):
             np.testing.assert_allclose(o, want, rtol=1e-11, atol=1e-12)
 
 
+def check_rows_match_full(ref):
+    """Row-sampled prefill gives exactly the full-layer result at those rows."""
+    q, k, v, sink = _rand_prefill(21, B=2, n=30, hq=4, hkv=2)
+    for window in (7, 0):
+        o, lse = ref.prefill(q, k, v, sink, window, 1e7, 8)
+        rows = [(1, 3, 29), (0, 0, 0), (0, 2, 17), (1, 1, 6)]
+        o2, l2 = ref.prefill(q, k, v, sink, window, 1e7, 8, rows=rows)
+        for r, (b, h, i) in enumerate(rows):
+            np.testing.assert_array_equal(o2[r], o[b, i, h])
+            assert l2[r] == lse[b, h, i]
+
+
 def check_window_ge_n_is_causal(ref):
     """§2: SWA differs from global attention only in the range of j, so a
     window >= n gives full causal attention (torch SDPA is_causal)."""
@@ -361,6 +373,7 @@ ALL_CHECKS = [
     check_sink_limits,
     check_against_sdpa,
     check_window_ge_n_is_causal,
+    check_rows_match_full,
     check_window_membership,
     check_receptive_field,
     check_rope_against_hf,

@@ -1,0 +1,122 @@
+"""Host-side checks of the C ABI (no GPU work): the library loads, exports every
+symbol the header declares, and rejects bad arguments before any launch."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from hybrid_sliding_window_sink_b200 import _lib
+from hybrid_sliding_window_sink_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mimo_attn.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    build()
+    return _lib.lib()
+
+
+def _declared():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(mimo_\w+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = _declared()
+    assert set(names) == set(_lib.EXPORTS)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings_and_version(L):
+    for code in range(8):
+        s = L.mimo_status_string(code).decode()
+        assert s and s != "unknown status"
+    assert L.mimo_status_string(99).decode() == "unknown status"
+    assert L.mimo_attn_version() >= 100
+
+
+def _shape(**kw):
+    base = dict(batch=1, seqlen=64, hq=8, hkv=1, dqk=192, dv=128, softmax_scale=0.0)
+    base.update(kw)
+    return _lib.make_shape(base["batch"], base["seqlen"], base["hq"], base["hkv"], base["dqk"],
+                           base["dv"], base["softmax_scale"])
+
+
+P = ctypes.c_void_p
+GOOD = P(0x10000)   # never dereferenced: every case below fails validation first
+
+
+def _prefill(L, shape, q=GOOD, k=GOOD, v=GOOD, out=GOOD, sink=None, lse=None, window=128,
+             theta=1e4, rot=64):
+    return L.mimo_attn_prefill(ctypes.byref(shape), q, k, v, sink, window, theta, rot, out, lse, None)
+
+
+def test_prefill_rejects_before_launch(L):
+    assert L.mimo_attn_prefill(None, GOOD, GOOD, GOOD, None, 128, 1e4, 64, GOOD, None, None) == 1
+    assert _prefill(L, _shape(), q=None) == 1
+    assert _prefill(L, _shape(), out=None) == 1
+    assert _prefill(L, _shape(seqlen=0)) == 2
+    assert _prefill(L, _shape(batch=0)) == 2
+    assert _prefill(L, _shape(hq=6, hkv=4)) == 2
+    assert _prefill(L, _shape(hq=64, hkv=2)) == 3          # group 32
+    assert _prefill(L, _shape(hq=12, hkv=4)) == 3          # group 3
+    assert _prefill(L, _shape(dqk=128)) == 3
+    assert _prefill(L, _shape(dv=192)) == 3
+    assert _prefill(L, _shape(softmax_scale=float("nan"))) == 2
+    assert _prefill(L, _shape(), rot=-2) == 2
+    assert _prefill(L, _shape(), rot=200) == 2
+    assert _prefill(L, _shape(), rot=40) == 3
+    assert _prefill(L, _shape(), theta=0.0) == 2
+    assert _prefill(L, _shape(), theta=float("inf")) == 2
+    assert _prefill(L, _shape(), q=P(0x10008)) == 4
+    assert _prefill(L, _shape(), out=P(0x10004)) == 4
+    assert _prefill(L, _shape(), sink=P(0x10002)) == 4
+
+
+def _decode(L, shape, kind=0, cap=128, stride=128, lengths=GOOD, q=GOOD, ws=None, nbytes=0):
+    return L.mimo_attn_decode(ctypes.byref(shape), q, GOOD, GOOD, kind, cap, stride, lengths, None,
+                              GOOD, None, ws, nbytes, None)
+
+
+def test_decode_rejects_before_launch(L):
+    s = _shape(hq=64, hkv=8)
+    assert _decode(L, s, kind=5) == 2
+    assert _decode(L, s, lengths=None) == 1
+    assert _decode(L, s, q=None) == 1
+    assert _decode(L, s, cap=0) == 2
+    assert _decode(L, s, cap=256, stride=128) == 2
+    assert _decode(L, s, q=P(0x10001)) == 4
+    assert _decode(L, s, lengths=P(0x10002)) == 4
+    assert _decode(L, _shape(hq=64, hkv=8, dqk=64)) == 3
+
+
+def test_sparse_rejects_before_launch(L):
+    s = _shape(hq=64, hkv=4)
+    f = L.mimo_attn_sparse
+    assert f(ctypes.byref(s), GOOD, GOOD, GOOD, 4096, 4096, GOOD, 128, None, 16, None, GOOD, None,
+             None, 0, None) == 1
+    assert f(ctypes.byref(s), GOOD, GOOD, GOOD, 4096, 4096, GOOD, -1, GOOD, 16, None, GOOD, None,
+             None, 0, None) == 2
+    assert f(ctypes.byref(s), GOOD, GOOD, GOOD, 4096, 4096, GOOD, 128, GOOD, -3, None, GOOD, None,
+             None, 0, None) == 2
+
+
+def test_workspace_size_plans(L):
+    # ring of 128 slots: one chunk per (b, g), finalised in place, no workspace
+    assert _lib.workspace_size(64, 64, 8, op=_lib.MIMO_OP_DECODE, kind=_lib.MIMO_CACHE_RING,
+                               capacity=128) == 0
+    # long linear cache: split-KV partials (m, l) + o per chunk
+    n = _lib.workspace_size(64, 64, 4, op=_lib.MIMO_OP_DECODE, kind=_lib.MIMO_CACHE_LINEAR,
+                            capacity=131072)
+    assert n > 0 and n % 4 == 0
+    nsp = _lib.workspace_size(8, 64, 4, op=_lib.MIMO_OP_SPARSE, capacity=262144, recent=128,
+                              n_sel=1024)
+    assert nsp > 0
+    assert _lib.workspace_size(8, 64, 4, op=7, capacity=10) == 0
+    assert _lib.workspace_size(8, 64, 4, op=_lib.MIMO_OP_SPARSE, capacity=10, recent=-1) == 0

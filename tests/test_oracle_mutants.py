@@ -27,7 +27,8 @@ MUTANTS = {
     "rope interleaved partner": ("x2 = x[..., half:rot_dims]", "x2 = np.roll(x[..., :rot_dims], -1, axis=-1)[..., :half]"),
     "scale ignored": ("return 1.0 / math.sqrt(d) if not scale else float(scale)", "return 1.0"),
     "gqa map modulo": ("        g = h // group\n        keys = window_keys", "        g = h % Hkv\n        keys = window_keys"),
-    "scores against V": ("a = (K[keys] @ _f64(q_i)) * scale\n    s, lse", "a = (K[keys][:, :1] @ _f64(q_i)[:1]) * scale\n    s, lse"),
+    "scores on a truncated dot product": ("a = (Kj @ _f64(q_i)) * scale", "a = (Kj[:, :1] @ _f64(q_i)[:1]) * scale"),
+    "values gathered from keys": ("o = s @ Vj", "o = s @ Kj[:, :Vj.shape[1]]"),
     "ring slots off by one": ("return np.arange(min(L, capacity), dtype=np.int64)",
                               "return np.arange(min(L, capacity) - 1, dtype=np.int64)"),
     "sparse window misses newest": ("win = np.arange(max(0, L - recent), L, dtype=np.int64)",

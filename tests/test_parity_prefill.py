@@ -1,0 +1,156 @@
+"""Prefill parity: the sm_100a kernel through the C ABI against the float64 oracle."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from hybrid_sliding_window_sink_b200 import _lib, workloads as wl
+from oracle import ref
+from parity_util import compare
+
+pytestmark = pytest.mark.gpu
+
+
+def _run_and_compare(inp, window, theta, rot, dev, what, scale=0.0):
+    q, k, v, sink = (inp["q"].to(dev), inp["k"].to(dev), inp["v"].to(dev),
+                     None if inp["sink"] is None else inp["sink"].to(dev))
+    out, lse = _lib.prefill(q, k, v, sink, window=window, rope_theta=theta, rot_dims=rot,
+                            softmax_scale=scale)
+    torch.cuda.synchronize()
+    assert _lib.last_device_error() == 0
+    o_ref, l_ref = ref.prefill(wl.to_f64(inp["q"]), wl.to_f64(inp["k"]), wl.to_f64(inp["v"]),
+                               None if inp["sink"] is None else wl.to_f64(inp["sink"]),
+                               window, theta, rot, scale=scale or None)
+    return compare(wl.to_f64(out), o_ref, wl.to_f64(lse), l_ref, what)
+
+
+def test_tiny_swa_config(cuda_device):
+    """Tiny SWA+sink prefill: n=1024, 8 Q / 1 KV heads, W=128, RoPE 64 dims theta 1e4."""
+    c = wl.TINY_SWA_PREFILL
+    inp = wl.case_prefill_inputs(c)
+    _run_and_compare(inp, c.window, c.theta, wl.ROT_DIMS, cuda_device, c.name)
+
+
+@pytest.mark.parametrize("n,hq,hkv,window,sink,rot", [
+    (16, 8, 1, 128, False, 0),        # one tile, no RoPE, no sink
+    (16, 8, 1, 128, True, 64),
+    (1, 8, 1, 128, True, 64),         # single row
+    (37, 8, 1, 5, True, 64),          # ragged, tiny window
+    (300, 8, 1, 128, True, 64),       # several row blocks, ragged tail
+    (300, 16, 1, 128, True, 64),      # group 16 (8 positions per block)
+    (300, 8, 2, 1, True, 64),         # window 1: only the diagonal
+    (300, 8, 2, 299, True, 64),       # window n-1
+    (200, 4, 1, 128, True, 64),       # group 4: P + W - 1 > 144, multi-tile SWA
+    (200, 2, 2, 17, True, 16),        # group 1, 128 positions per block
+])
+def test_swa_shapes(cuda_device, n, hq, hkv, window, sink, rot):
+    inp = wl.prefill_inputs(1, n, hq, hkv, seed=100 + n + hq + window, with_sink=sink)
+    _run_and_compare(inp, window, wl.SWA_THETA, rot, cuda_device, f"swa n={n} {hq}/{hkv} W={window}")
+
+
+@pytest.mark.parametrize("B,n,hq,hkv,rot,k_scale", [
+    (1, 129, 8, 1, 64, 0.5),
+    (1, 600, 16, 1, 64, 0.5),         # GA heads 16 per KV head, several key tiles
+    (2, 300, 8, 2, 64, 1.0),          # batch 2
+    (1, 257, 4, 1, 128, 1.0),         # group 4
+    (1, 130, 2, 2, 192, 1.0),         # group 1, full-width RoPE
+    (1, 200, 8, 1, 0, 1.0),           # no RoPE
+])
+def test_ga_shapes(cuda_device, B, n, hq, hkv, rot, k_scale):
+    inp = wl.prefill_inputs(B, n, hq, hkv, seed=200 + n + hq, k_scale=k_scale)
+    _run_and_compare(inp, 0, wl.GA_THETA, rot, cuda_device, f"ga B={B} n={n} {hq}/{hkv}")
+
+
+def test_window_ge_n_equals_ga(cuda_device):
+    """W >= n is full causal attention: same result as window = 0, bit for bit."""
+    inp = wl.prefill_inputs(1, 200, 8, 1, seed=7)
+    q, k, v, s = (inp[x].to(cuda_device) for x in ("q", "k", "v", "sink"))
+    a, la = _lib.prefill(q, k, v, s, window=200, rope_theta=1e4, rot_dims=64)
+    b, lb = _lib.prefill(q, k, v, s, window=0, rope_theta=1e4, rot_dims=64)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b) and torch.equal(la, lb)
+
+
+def test_sink_closed_form_on_gpu(cuda_device):
+    """V = 1 makes o the total weight S/(e^sink + S) = 1 - exp(sink - lse) (no oracle)."""
+    inp = wl.prefill_inputs(1, 300, 8, 1, seed=9)
+    v1 = torch.ones_like(inp["v"]).to(cuda_device)
+    q, k, s = (inp[x].to(cuda_device) for x in ("q", "k", "sink"))
+    out, lse = _lib.prefill(q, k, v1, s, window=128, rope_theta=1e4, rot_dims=64)
+    torch.cuda.synchronize()
+    want = 1.0 - torch.exp(s.double()[None, :, None] - lse.double())      # [1, Hq, n]
+    got = out.double()[..., 0].permute(0, 2, 1)
+    assert float((got - want).abs().max()) < 1e-2
+
+
+def test_large_and_missing_sink(cuda_device):
+    inp = wl.prefill_inputs(1, 150, 8, 1, seed=11)
+    inp["sink"] = torch.full((8,), 30.0)
+    _run_and_compare(inp, 128, 1e4, 64, cuda_device, "sink 30")
+    inp["sink"] = torch.full((8,), -1e4)
+    _run_and_compare(inp, 128, 1e4, 64, cuda_device, "sink -1e4")
+    inp["sink"] = None
+    _run_and_compare(inp, 0, 1e7, 64, cuda_device, "GA no sink")
+
+
+def test_deterministic_and_guarded(cuda_device):
+    """Two runs give identical bits; writes stay inside out / lse (guard bands)."""
+    inp = wl.prefill_inputs(1, 333, 16, 1, seed=12)
+    q, k, v, s = (inp[x].to(cuda_device) for x in ("q", "k", "v", "sink"))
+    guard = 4096
+    o_buf = torch.full((guard * 2 + 333 * 16 * 128,), 7.0, dtype=torch.bfloat16, device=cuda_device)
+    l_buf = torch.full((guard * 2 + 16 * 333,), 7.0, dtype=torch.float32, device=cuda_device)
+    out = o_buf[guard:guard + 333 * 16 * 128].view(1, 333, 16, 128)
+    lse = l_buf[guard:guard + 16 * 333].view(1, 16, 333)
+    _lib.prefill(q, k, v, s, window=128, rope_theta=1e4, rot_dims=64, out=out, lse=lse)
+    first = (out.clone(), lse.clone())
+    _lib.prefill(q, k, v, s, window=0, rope_theta=1e7, rot_dims=64, out=out, lse=lse)
+    _lib.prefill(q, k, v, s, window=128, rope_theta=1e4, rot_dims=64, out=out, lse=lse)
+    torch.cuda.synchronize()
+    assert torch.equal(first[0], out) and torch.equal(first[1], lse)
+    assert bool((o_buf[:guard] == 7.0).all()) and bool((o_buf[-guard:] == 7.0).all())
+    assert bool((l_buf[:guard] == 7.0).all()) and bool((l_buf[-guard:] == 7.0).all())
+
+
+def _sample_rows(n, nrand, seed, tile_rows=(16, 8)):
+    r = np.random.default_rng(seed)
+    rows = set(range(0, 96)) | set(range(n - 96, n))
+    for t in (127, 128, 129, 143, 144, 145, 255, 256):
+        rows |= {t - 1, t, t + 1}
+    rows |= set(r.choice(n, nrand, replace=False).tolist())
+    return sorted(x for x in rows if 0 <= x < n)
+
+
+@pytest.mark.parametrize("case,nrand,heads", [
+    (wl.SWA_PREFILL, 256, None),
+    (wl.GA_PREFILL, 24, 16),
+])
+def test_full_size_sampled(cuda_device, case, nrand, heads):
+    """Full-size configurations, exactly as the benchmark launches them, against the
+    oracle on sampled rows (start, end, tile boundaries, seeded random rows)."""
+    inp = wl.case_prefill_inputs(case, device=cuda_device)
+    out, lse = _lib.prefill(inp["q"], inp["k"], inp["v"], inp["sink"], window=case.window,
+                            rope_theta=case.theta, rot_dims=wl.ROT_DIMS)
+    torch.cuda.synchronize()
+    assert _lib.last_device_error() == 0
+    n = case.seqlen
+    pos = _sample_rows(n, nrand, case.seed)
+    hs = list(range(case.hq)) if heads is None else sorted(
+        np.random.default_rng(case.seed + 1).choice(case.hq, heads, replace=False).tolist())
+    # the oracle receives the exact bf16 values: the sampled query rows and all of K, V
+    qs = wl.to_f64(inp["q"][0, pos])                                  # [len(pos), Hq, 192]
+    rows = [(0, h, i) for i in pos for h in hs]
+    q_rows = np.stack([qs[a, h] for a in range(len(pos)) for h in hs])
+    o_ref, l_ref = ref.prefill_rows(q_rows, wl.to_f64(inp["k"]), wl.to_f64(inp["v"]),
+                                    wl.to_f64(inp["sink"]), case.window, case.theta, wl.ROT_DIMS,
+                                    rows, case.hq)
+    og = wl.to_f64(out[0, pos])                                       # [len(pos), Hq, 128]
+    lg = wl.to_f64(lse[0][:, pos])                                    # [Hq, len(pos)]
+    o_gpu = np.stack([og[a, h] for a in range(len(pos)) for h in hs])
+    l_gpu = np.array([lg[h, a] for a in range(len(pos)) for h in hs])
+    compare(o_gpu, o_ref, l_gpu, l_ref, case.name)
+    assert torch.isfinite(out).all() and torch.isfinite(lse).all()
+    del inp, out, lse
+    torch.cuda.empty_cache()
