@@ -65,7 +65,7 @@ class ClockSampler:
             self.out = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", uuid, f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=self.out, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -143,6 +143,12 @@ def timed(fn, steps, warmup, stream, flush=None):
     torch.cuda.synchronize()
     D.barrier()
     return e0.elapsed_time(e1)
+
+
+def timed_stream(fn, steps, warmup, stream):
+    """``timed`` with the events recorded on ``stream`` (the stream the work runs on)."""
+    with torch.cuda.stream(stream):
+        return timed(fn, steps, warmup, stream)
 
 
 def roofline_hbm(bytes_per_launch, ms_per_launch, peaks, tag, traffic=None):
@@ -325,13 +331,25 @@ def bench_sparse(steps, warmup, peaks, tag, dev, stream, calls=16):
             _lib.sparse(q, base["k_cache"], base["v_cache"], base["lengths"], sel, base["sink"],
                         recent=c.recent, out=out, lse=lse, workspace=ws, stream=stream)
 
+    # capture on a side stream (graphs cannot be captured on the legacy default stream)
+    cap_stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize()
     graph = torch.cuda.CUDAGraph()
-    calls_fn()   # loads the library and warms caches outside capture
+    with torch.cuda.stream(cap_stream):
+        calls_fn_s = lambda: [  # noqa: E731
+            _lib.sparse(q, base["k_cache"], base["v_cache"], base["lengths"], sel, base["sink"],
+                        recent=c.recent, out=out, lse=lse, workspace=ws, stream=cap_stream)
+            for (q, sel, out, lse, ws) in sets]
+        calls_fn_s()   # loads the library and warms caches outside capture
+        cap_stream.synchronize()
+        with torch.cuda.graph(graph, stream=cap_stream):
+            calls_fn_s()
     torch.cuda.synchronize()
-    with torch.cuda.graph(graph, stream=stream):
-        calls_fn()
-    ms = timed(graph.replay, steps, warmup, stream)
+
+    def replay():
+        graph.replay()
+
+    ms = timed_stream(replay, steps, warmup, cap_stream)
     per_call_bytes = (c.batch * c.hkv * (c.recent + c.n_sel) * (wl.DQK + wl.DV) * 2
                       + c.batch * c.hkv * c.n_sel * 4 + c.batch * c.hq * (wl.DQK + wl.DV) * 2
                       + c.batch * c.hq * 4 + c.hq * 4 + c.batch * 4)
@@ -348,7 +366,7 @@ def bench_sparse(steps, warmup, peaks, tag, dev, stream, calls=16):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=500)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="mimo", choices=["mimo", "reference"])
     ap.add_argument("--only-main", action="store_true", help="skip the extra workloads")

@@ -22,7 +22,8 @@
 //   warp 1     allocates 512 TMEM columns; one thread issues tcgen05.mma:
 //              S = Q K^T into a double-buffered TMEM S tile, O += P V into TMEM O.
 //   warps 2-5  compute group: RoPE of Q and K tiles in shared memory (fp64 angle
-//              reduction, fp32 sin/cos), sink-seeded online softmax from TMEM S,
+//              reduction, fp32 sin/cos, rotated dims kept as f16), sink-seeded
+//              online softmax from TMEM S,
 //              P (bf16) to shared memory, O rescale in TMEM, epilogue O / l -> bf16.
 // Every wait is bounded in time; on a timeout all roles leave their loops, the
 // producer and MMA thread wait (bounded) for their in-flight work, TMEM is freed
@@ -69,6 +70,7 @@ struct PfCfg {
   static constexpr int S1_COL = (BN + 31) / 32 * 32;
   static constexpr int O_COL = (S1_COL + BN + 31) / 32 * 32;
   static constexpr uint32_t IDESC_S = idesc_bf16(128, BN, 0, 0);
+  static constexpr uint32_t IDESC_S_F16 = idesc_f16kind(128, BN, 0, 0, 1);   // rotated dims
   static constexpr uint32_t IDESC_PV = idesc_bf16(128, 128, 0, 1);
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N");
   static_assert(K_CHUNK % 1024 == 0, "swizzle atoms");
@@ -87,6 +89,10 @@ enum : int {
 // Rotates dims [0, rot) of one tile row in place (rotate-half pairing (d, d + rot/2)).
 // The row lives in 64-dim chunks of `chunk_bytes`, 128 bytes per row, with the
 // 16-byte units XOR-swizzled by (row & 7) as the 128-byte TMA swizzle writes them.
+// Inputs are bf16; the rotated values are written back as f16 (11 significant bits
+// instead of 8), and the QK^T k-steps over [0, rot) run as f16 x f16 MMAs. Rounding
+// the rotated q and k to bf16 would perturb the scores by ~1e-3 (the size of the
+// LSE tolerance); f16 cuts that eightfold. Values are clamped to the f16 range.
 __device__ __forceinline__ void rope_row(uint32_t base, int chunk_bytes, int row, int pos, int rot,
                                          const double* invf) {
   const int nun = rot >> 4;   // 8-dim units per half
@@ -115,8 +121,8 @@ __device__ __forceinline__ void rope_row(uint32_t base, int chunk_bytes, int row
         r1[h] = v1 * c - v2 * s;
         r2[h] = v2 * c + v1 * s;
       }
-      x[e2] = pack_bf16(r1[0], r1[1]);
-      y[e2] = pack_bf16(r2[0], r2[1]);
+      x[e2] = pack_f16_sat(r1[0], r1[1]);
+      y[e2] = pack_f16_sat(r2[0], r2[1]);
     }
     st_shared_v4(a1, x[0], x[1], x[2], x[3]);
     st_shared_v4(a2, y[0], y[1], y[2], y[3]);
@@ -254,7 +260,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             const uint32_t off = (kk & 3) * 32u;   // 16-dim step inside the 128-byte row
             const uint64_t a = smem_desc(sQ + (kk >> 2) * C::Q_CHUNK + off, 16, 1024);
             const uint64_t bd = smem_desc(sK + (kk >> 2) * C::K_CHUNK + off, 16, 1024);
-            umma_ss(d, a, bd, C::IDESC_S, kk > 0 ? 1u : 0u);
+            const uint32_t idesc = kk * 16 < p.rot_dims ? C::IDESC_S_F16 : C::IDESC_S;
+            umma_ss(d, a, bd, idesc, kk > 0 ? 1u : 0u);
           }
           umma_commit(bar(kBarKEmpty0 + ks));
           umma_commit(bar(kBarSFull0 + sb));
