@@ -25,7 +25,8 @@ STATUS = {0: "MIMO_OK", 1: "MIMO_ERR_NULL", 2: "MIMO_ERR_SHAPE", 3: "MIMO_ERR_UN
           4: "MIMO_ERR_ALIGN", 5: "MIMO_ERR_WORKSPACE", 6: "MIMO_ERR_CUDA", 7: "MIMO_ERR_DEVICE"}
 
 #: Every symbol include/mimo_attn.h declares.
-EXPORTS = ("mimo_attn_prefill", "mimo_attn_decode", "mimo_attn_sparse", "mimo_attn_workspace_size",
+EXPORTS = ("mimo_attn_prefill", "mimo_attn_decode", "mimo_attn_sparse", "mimo_attn_sparse_noalloc",
+           "mimo_attn_workspace_size",
            "mimo_attn_check_indices", "mimo_attn_last_device_error", "mimo_status_string",
            "mimo_attn_version")
 
@@ -62,6 +63,7 @@ def lib():
     L.mimo_attn_prefill.argtypes = [SP, P, P, P, P, I, F, I, P, P, P]
     L.mimo_attn_decode.argtypes = [SP, P, P, P, I, I, LL, P, P, P, P, P, SZ, P]
     L.mimo_attn_sparse.argtypes = [SP, P, P, P, I, LL, P, I, P, I, P, P, P, P, SZ, P]
+    L.mimo_attn_sparse_noalloc.argtypes = [SP, P, P, P, I, LL, P, I, P, I, P, P, P, P]
     L.mimo_attn_workspace_size.argtypes = [SP, I, I, I, I, I]
     L.mimo_attn_workspace_size.restype = SZ
     L.mimo_attn_check_indices.argtypes = [SP, P, P, I, I, I, P, P]
@@ -71,7 +73,8 @@ def lib():
     L.mimo_status_string.restype = ctypes.c_char_p
     L.mimo_attn_version.argtypes = []
     L.mimo_attn_version.restype = I
-    for fn in ("mimo_attn_prefill", "mimo_attn_decode", "mimo_attn_sparse", "mimo_attn_check_indices"):
+    for fn in ("mimo_attn_prefill", "mimo_attn_decode", "mimo_attn_sparse", "mimo_attn_sparse_noalloc",
+               "mimo_attn_check_indices"):
         getattr(L, fn).restype = I
     _LIB = L
     return L

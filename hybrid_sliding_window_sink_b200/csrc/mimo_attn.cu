@@ -399,3 +399,52 @@ const char* mimo_status_string(mimo_status st) {
 int mimo_attn_version(void) { return 100; }
 
 }  // extern "C"
+
+// ============================================================== allocation-free sparse decode
+// The split-KV partials of mimo_attn_sparse_noalloc live in this library-owned array
+// instead of a caller workspace. Host code must not pass the symbol itself to a kernel:
+// on the host it names a stand-in, not device memory. The device address is looked up
+// once per device (with that device current) and cached.
+static __device__ __align__(256) unsigned char g_sparse_noalloc_scratch[MIMO_SPARSE_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+std::atomic<void*> g_noalloc_ptr[kMaxDevices];
+
+void* noalloc_scratch(int dev) {
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
+  void* p = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+  if (p) return p;
+  void* addr = nullptr;
+  if (cudaGetSymbolAddress(&addr, g_sparse_noalloc_scratch) != cudaSuccess || addr == nullptr) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  g_noalloc_ptr[dev].store(addr, std::memory_order_release);
+  return addr;
+}
+}  // namespace
+
+extern "C" mimo_status mimo_attn_sparse_noalloc(const mimo_shape* s, const void* q,
+                                                const void* k_cache, const void* v_cache,
+                                                int cache_capacity, long long seq_stride_tokens,
+                                                const int* lengths, int recent, const int* sel_idx,
+                                                int n_sel, const float* sink, void* out, float* lse,
+                                                void* stream) {
+  mimo_status e = check_heads(s);
+  if (e != MIMO_OK) return e;
+  if (cache_capacity < 1 || recent < 0 || n_sel < 0) return MIMO_ERR_SHAPE;
+  const int dev = current_device();
+  if (dev < 0) return MIMO_ERR_CUDA;
+  const size_t need =
+      plan_decode(s, mimo::kModeSparse, cache_capacity, recent, n_sel, sm_count_for(dev)).bytes;
+  if (need > MIMO_SPARSE_NOALLOC_SCRATCH_BYTES) return MIMO_ERR_WORKSPACE;
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
+  if (need > 0) {
+    ws = noalloc_scratch(dev);
+    if (!ws) return MIMO_ERR_CUDA;
+    ws_bytes = MIMO_SPARSE_NOALLOC_SCRATCH_BYTES;
+  }
+  return run_decode(s, mimo::kModeSparse, q, k_cache, v_cache, cache_capacity, seq_stride_tokens,
+                    lengths, recent, sel_idx, n_sel, sink, out, lse, ws, ws_bytes, stream);
+}

@@ -32,8 +32,9 @@
  *  - Supported head dims: head_dim_qk = 192, head_dim_v = 128. n_q_heads must be a
  *    multiple of n_kv_heads with group n_q_heads / n_kv_heads in {1, 2, 4, 8, 16};
  *    query head h reads KV head h / group (contiguous groups).
- *  - Thread safety: calls may be made from several host threads; the only shared
- *    mutable state is the device error word read by mimo_attn_last_device_error.
+ *  - Thread safety: calls may be made from several host threads; the shared mutable
+ *    state is the device error word read by mimo_attn_last_device_error and the scratch
+ *    array of mimo_attn_sparse_noalloc (see there).
  */
 #ifndef MIMO_ATTN_H
 #define MIMO_ATTN_H
@@ -151,6 +152,37 @@ mimo_status mimo_attn_sparse(const mimo_shape* shape, const void* q, const void*
  * on the current device (0 when none is needed). Returns 0 for invalid arguments. */
 size_t mimo_attn_workspace_size(const mimo_shape* shape, int op, int cache_kind,
                                 int cache_capacity, int recent, int n_sel);
+
+/* Fixed size of the library-owned scratch array used by mimo_attn_sparse_noalloc (8 MiB). */
+#define MIMO_SPARSE_NOALLOC_SCRATCH_BYTES 8388608u
+
+/*
+ * Allocation-free variant of mimo_attn_sparse. The paper has no counterpart: this is a
+ * deployment convenience of this library.
+ *
+ * Who needs it: callers that cannot allocate device memory when they call attention,
+ * e.g. a serving loop whose KV-cache pools reserve nearly all of HBM up front (a late
+ * cudaMalloc would fail or force evictions), or a plug-in inside a host framework that
+ * owns every device allocation and forbids direct cudaMalloc / cudaFree (cudaFree also
+ * synchronises the whole device). They pass inputs and outputs only; the split-KV
+ * partials go to a static device array of MIMO_SPARSE_NOALLOC_SCRATCH_BYTES that the
+ * library holds on every GPU that loads it, until the process exits.
+ *
+ * Arguments and results are those of mimo_attn_sparse without workspace. Returns
+ * MIMO_ERR_WORKSPACE, with nothing launched, when these sizes need more scratch than
+ * the array holds (mimo_attn_workspace_size(shape, MIMO_OP_SPARSE, ...) larger than
+ * MIMO_SPARSE_NOALLOC_SCRATCH_BYTES). The first call on a device looks up the array's
+ * device address with that device current (a host-side query, no allocation); make that
+ * first call before any stream capture. All calls share the one array: two calls whose
+ * kernels overlap on the GPU (different streams, no ordering between them) race on it
+ * and give wrong results; order them on one stream. No part of the array needs to start
+ * at zero: each call writes every partial it later reads.
+ */
+mimo_status mimo_attn_sparse_noalloc(const mimo_shape* shape, const void* q, const void* k_cache,
+                                     const void* v_cache, int cache_capacity,
+                                     long long seq_stride_tokens, const int* lengths, int recent,
+                                     const int* sel_idx, int n_sel, const float* sink, void* out,
+                                     float* lse, void* stream);
 
 /* Debug check of sparse-decode preconditions, on `stream`: counts, into the device
  * word *d_violations (which the caller zeroes first), every (b, g) row whose
