@@ -124,12 +124,22 @@ def decode_layer_bytes(lengths, hq, hkv, kind, cap):
 
 
 # ----------------------------------------------------------------------------- timing
+class DeviceError(RuntimeError):
+    pass
+
+
 def timed(fn, steps, warmup, stream, flush=None):
     """Run ``warmup`` untimed steps, then time exactly ``steps`` with CUDA events on
-    ``stream``, bracketed by barrier + synchronize. Returns elapsed ms of this rank."""
+    ``stream``, bracketed by barrier + synchronize. Returns elapsed ms of this rank.
+    Raises DeviceError (before timing) if a warm-up step set the library's device error
+    word, so that a broken kernel is not timed."""
+    from hybrid_sliding_window_sink_b200 import _lib
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize()
+    err = _lib.last_device_error()
+    if err:
+        raise DeviceError(f"device error word {err} set during warm-up")
     D.barrier()
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)

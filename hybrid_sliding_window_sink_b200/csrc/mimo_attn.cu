@@ -14,10 +14,17 @@
 #include "ptx.cuh"
 #include "decode.cuh"
 #include "prefill.cuh"
+#include "prefill_swa.cuh"
 
 namespace mimo {
 __device__ unsigned g_device_error = 0;
 }
+
+#ifdef MIMO_TRACE
+// Debug builds only: device buffer that receives per-phase timestamps of the prefill kernels.
+static unsigned long long* g_trace = nullptr;
+extern "C" void mimo_attn_debug_set_trace(void* p) { g_trace = static_cast<unsigned long long*>(p); }
+#endif
 
 namespace {
 
@@ -139,11 +146,37 @@ mimo_status launch_prefill(const mimo_shape* s, const void* q, const void* k, co
   return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ERR_CUDA;
 }
 
+// SWA layer with 8 query heads per KV head, W <= 129, rot_dims <= 64: the ring kernel.
+mimo_status launch_prefill_swa(const mimo_shape* s, const void* q, const void* k, const void* v,
+                               PrefillParams prm, int sms, cudaStream_t st) {
+  using L = mimo::SwaLayout;
+  CUtensorMap tq, tk, tv;
+  const uint64_t n = static_cast<uint64_t>(s->seqlen), B = static_cast<uint64_t>(s->batch);
+  if (!make_tmap(&tq, q, mimo::kDQK, s->n_q_heads, n, B, mimo::kSwaG, mimo::kSwaP) ||
+      !make_tmap(&tk, k, mimo::kDQK, s->n_kv_heads, n, B, 1, 16) ||
+      !make_tmap(&tv, v, mimo::kDV, s->n_kv_heads, n, B, 1, 16))
+    return MIMO_ERR_CUDA;
+  if (cudaFuncSetAttribute(mimo::prefill_swa_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           L::SMEM) != cudaSuccess) {
+    cudaGetLastError();
+    return MIMO_ERR_CUDA;
+  }
+  prm.n_qtiles = (s->seqlen + mimo::kSwaP - 1) / mimo::kSwaP;
+  const long long work = static_cast<long long>(s->batch) * s->n_kv_heads * prm.n_qtiles;
+  if (work > 0x7fffffffLL) return MIMO_ERR_UNSUPPORTED;
+  prm.num_work = static_cast<int>(work);
+  const int grid = prm.num_work < sms ? prm.num_work : sms;
+  mimo::prefill_swa_kernel<<<grid, mimo::kSwaThreads, L::SMEM, st>>>(tq, tk, tv, prm);
+  return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ERR_CUDA;
+}
+
 template <int G>
 mimo_status prefill_group(const mimo_shape* s, const void* q, const void* k, const void* v,
                           const PrefillParams& prm, int sms, cudaStream_t st) {
   constexpr int P = 128 / G;
   const bool swa = prm.window > 0 && prm.window < s->seqlen;
+  if (G == mimo::kSwaG && swa && prm.window <= 129 && prm.rot_dims <= 64)
+    return launch_prefill_swa(s, q, k, v, prm, sms, st);
   // one 144-key tile covers the whole window of a row block when P + W - 1 <= 144
   if (swa && P + prm.window - 1 <= 144) return launch_prefill<G, 144, 1>(s, q, k, v, prm, sms, st);
   return launch_prefill<G, 128, 2>(s, q, k, v, prm, sms, st);
@@ -305,6 +338,9 @@ mimo_status mimo_attn_prefill(const mimo_shape* s, const void* q, const void* k,
   prm.scale_log2 = scale_log2_of(s);
   prm.err = device_error_ptr(dev);
   if (!prm.err) return MIMO_ERR_CUDA;
+#ifdef MIMO_TRACE
+  prm.trace = g_trace;
+#endif
   const int sms = sm_count_for(dev);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   switch (s->n_q_heads / s->n_kv_heads) {

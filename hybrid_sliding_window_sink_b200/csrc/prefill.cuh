@@ -47,6 +47,7 @@ struct PrefillParams {
   float scale_log2;        // softmax scale * log2(e)
   int n_qtiles, num_work;
   unsigned* err;
+  unsigned long long* trace;   // debug timestamps (builds with -DMIMO_TRACE only), else null
 };
 
 template <int G, int BN, int NKS>

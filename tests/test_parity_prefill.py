@@ -50,6 +50,19 @@ def test_swa_shapes(cuda_device, n, hq, hkv, window, sink, rot):
     _run_and_compare(inp, window, wl.SWA_THETA, rot, cuda_device, f"swa n={n} {hq}/{hkv} W={window}")
 
 
+@pytest.mark.parametrize("B,n,hq,hkv,window,rot", [
+    (2, 3000, 16, 2, 128, 64),        # runs of row blocks crossing (b, kv-head) boundaries
+    (1, 5000, 8, 1, 129, 64),         # widest window of the ring kernel
+    (1, 2100, 64, 8, 100, 32),        # MiMo head layout, partial window, 32 rotated dims
+    (3, 700, 8, 1, 128, 0),           # no RoPE
+    (1, 2500, 16, 2, 7, 16),
+])
+def test_swa_ring_kernel(cuda_device, B, n, hq, hkv, window, rot):
+    """SWA layers with 8 query heads per KV head and W <= 129 (the K/V ring kernel)."""
+    inp = wl.prefill_inputs(B, n, hq, hkv, seed=150 + n + window)
+    _run_and_compare(inp, window, wl.SWA_THETA, rot, cuda_device, f"swa-ring B={B} n={n} W={window}")
+
+
 @pytest.mark.parametrize("B,n,hq,hkv,rot,k_scale", [
     (1, 129, 8, 1, 64, 0.5),
     (1, 600, 16, 1, 64, 0.5),         # GA heads 16 per KV head, several key tiles
