@@ -99,6 +99,25 @@ class ClockSampler:
                 "samples": len(sm), "reasons": sorted(reasons)}
 
 
+# ----------------------------------------------------------------------------- measured traffic
+def traffic_for(key, units):
+    """DRAM bytes of one launch from the ncu-measured bytes per unit (profiles/traffic.json),
+    or None when the kernel sources changed since the counters were taken."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f)[key]
+        h = hashlib.sha256()
+        for name in rec["sources"]:
+            with open(os.path.join(ROOT, "hybrid_sliding_window_sink_b200", "csrc", name), "rb") as f:
+                h.update(f.read())
+        if h.hexdigest()[:16] != rec["sha"]:
+            return None
+        return round(rec["bytes_per_unit"] * units)
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 # ----------------------------------------------------------------------------- algorithmic work
 def swa_pairs(n, window):
     if window <= 0 or window >= n:
@@ -304,7 +323,8 @@ def bench_decode_step(steps, warmup, peaks, tag, dev, stream):
         "value": round(total / (ms / steps * 1e-3) / 1e9, 1), "unit": "GB/s",
         "ms_per_step": round(ms / steps, 4), "bytes_per_step": total,
         "launches_per_step": 39 + 9 * 2,
-        "ga_layer": roofline_hbm(b_ga, ms_ga, peaks, tag),
+        "ga_layer": roofline_hbm(b_ga, ms_ga, peaks, tag,
+                                 traffic_for("decode_split_linear", int(sum(Ls)) * cg.hkv)),
         "swa_layer": roofline_hbm(b_swa, ms_swa, peaks, tag),
         "roofline": roofline_hbm(total, ms / steps, peaks, tag),
         "ms_ga_layer": round(ms_ga, 4), "ms_swa_layer": round(ms_swa, 5),
@@ -366,7 +386,9 @@ def bench_sparse(steps, warmup, peaks, tag, dev, stream, calls=16):
     ms_call = ms / (steps * calls)
     res = {"value": round(per_call_bytes / (ms_call * 1e-3) / 1e9, 1), "unit": "GB/s",
            "ms_per_call": round(ms_call, 5), "bytes_per_call": per_call_bytes, "calls_per_step": calls,
-           "launches_per_call": 2, "roofline": roofline_hbm(per_call_bytes, ms_call, peaks, tag),
+           "launches_per_call": 2,
+           "roofline": roofline_hbm(per_call_bytes, ms_call, peaks, tag,
+                                    traffic_for("decode_split_sparse", c.batch * c.hkv)),
            "graph": True}
     del graph, sets, base
     return res
@@ -442,7 +464,9 @@ def main():
         "config": {"workload": case.name, "global_batch": case.batch * world, "seq_len": case.seqlen,
                    "parallelism": f"dp{world} (independent problems per rank)",
                    "l2": "inputs larger than L2 (1.52 GB per step)"},
-        "roofline": roofline_hbm(bytes_, ms_step, peaks, tag),
+        "roofline": roofline_hbm(bytes_, ms_step, peaks, tag,
+                                 traffic_for("prefill_swa_kernel",
+                                             case.batch * case.hkv * -(-case.seqlen // 16))),
         "tensor": roofline_tensor(flops, ms_step, peaks["bf16_tflops"], tag),
         "gpu_launches": args.steps,
         "clocks": clk,
@@ -468,7 +492,8 @@ def main():
             wls["ga_prefill"] = {
                 "workload": wl.GA_PREFILL.name, "value": round(ga["flops"] / (ms_ga * 1e-3) / 1e12, 2),
                 "unit": "TFLOP/s", "ms_per_step": round(ms_ga, 4),
-                "roofline": roofline_tensor(ga["flops"], ms_ga, peaks["bf16_tflops"], tag),
+                "roofline": roofline_tensor(ga["flops"], ms_ga, peaks["bf16_tflops"], tag,
+                                            traffic_for("prefill_kernel_ga", wl.GA_PREFILL.seqlen)),
                 "device_error": ga["device_error"]}
             del ga
             torch.cuda.empty_cache()

@@ -32,6 +32,10 @@
  *  - Supported head dims: head_dim_qk = 192, head_dim_v = 128. n_q_heads must be a
  *    multiple of n_kv_heads with group n_q_heads / n_kv_heads in {1, 2, 4, 8, 16};
  *    query head h reads KV head h / group (contiguous groups).
+ *  - Precision: products of bf16 inputs are exact and accumulate in fp32. The RoPE-rotated
+ *    Q/K dims (prefill) are carried in f16 for their MMAs, and the SWA prefill kernel keeps
+ *    P and V in f16; inputs are therefore expected inside the f16 range (|x| < 65504) -
+ *    values outside it are clamped. Outputs are rounded to bf16, lse is fp32.
  *  - Thread safety: calls may be made from several host threads; the shared mutable
  *    state is the device error word read by mimo_attn_last_device_error and the scratch
  *    array of mimo_attn_sparse_noalloc (see there).
