@@ -15,6 +15,7 @@
 #include "decode.cuh"
 #include "prefill.cuh"
 #include "prefill_swa.cuh"
+#include "prefill_ga.cuh"
 
 namespace mimo {
 __device__ unsigned g_device_error = 0;
@@ -170,6 +171,32 @@ mimo_status launch_prefill_swa(const mimo_shape* s, const void* q, const void* k
   return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ERR_CUDA;
 }
 
+// Full causal prefix (GA layers) with 8 or 16 query heads per KV head, rot_dims <= 64:
+// two row blocks per work item share every K/V tile.
+template <int G>
+mimo_status launch_prefill_ga(const mimo_shape* s, const void* q, const void* k, const void* v,
+                              PrefillParams prm, int sms, cudaStream_t st) {
+  using L = mimo::GaLayout<G>;
+  CUtensorMap tq, tk, tv;
+  const uint64_t n = static_cast<uint64_t>(s->seqlen), B = static_cast<uint64_t>(s->batch);
+  if (!make_tmap(&tq, q, mimo::kDQK, s->n_q_heads, n, B, G, L::P) ||
+      !make_tmap(&tk, k, mimo::kDQK, s->n_kv_heads, n, B, 1, mimo::kGaBN) ||
+      !make_tmap(&tv, v, mimo::kDV, s->n_kv_heads, n, B, 1, mimo::kGaBN))
+    return MIMO_ERR_CUDA;
+  auto kern = mimo::prefill_ga_kernel<G>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM) != cudaSuccess) {
+    cudaGetLastError();
+    return MIMO_ERR_CUDA;
+  }
+  prm.n_qtiles = (s->seqlen + 2 * L::P - 1) / (2 * L::P);   // pairs of row blocks
+  const long long work = static_cast<long long>(s->batch) * s->n_kv_heads * prm.n_qtiles;
+  if (work > 0x7fffffffLL) return MIMO_ERR_UNSUPPORTED;
+  prm.num_work = static_cast<int>(work);
+  const int grid = prm.num_work < sms ? prm.num_work : sms;
+  kern<<<grid, mimo::kGaThreads, L::SMEM, st>>>(tq, tk, tv, prm);
+  return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ERR_CUDA;
+}
+
 template <int G>
 mimo_status prefill_group(const mimo_shape* s, const void* q, const void* k, const void* v,
                           const PrefillParams& prm, int sms, cudaStream_t st) {
@@ -177,6 +204,9 @@ mimo_status prefill_group(const mimo_shape* s, const void* q, const void* k, con
   const bool swa = prm.window > 0 && prm.window < s->seqlen;
   if (G == mimo::kSwaG && swa && prm.window <= 129 && prm.rot_dims <= 64)
     return launch_prefill_swa(s, q, k, v, prm, sms, st);
+  if constexpr (G == 8 || G == 16) {
+    if (!swa && prm.rot_dims <= 64) return launch_prefill_ga<G>(s, q, k, v, prm, sms, st);
+  }
   // one 144-key tile covers the whole window of a row block when P + W - 1 <= 144
   if (swa && P + prm.window - 1 <= 144) return launch_prefill<G, 144, 1>(s, q, k, v, prm, sms, st);
   return launch_prefill<G, 128, 2>(s, q, k, v, prm, sms, st);

@@ -76,6 +76,32 @@ def test_ga_shapes(cuda_device, B, n, hq, hkv, rot, k_scale):
     _run_and_compare(inp, 0, wl.GA_THETA, rot, cuda_device, f"ga B={B} n={n} {hq}/{hkv}")
 
 
+@pytest.mark.parametrize("B,n,hq,hkv,rot,k_scale,ramp", [
+    (2, 3000, 32, 2, 64, 0.5, False),  # 16 heads per KV head, more work items than SMs
+    (1, 1000, 64, 8, 64, 1.0, False),  # 8 heads per KV head
+    (1, 9, 16, 1, 64, 1.0, False),     # second row block wholly past the end, one key tile
+    (1, 24, 16, 1, 32, 1.0, False),    # second row block partly past the end
+    (3, 515, 16, 4, 0, 2.0, False),    # no RoPE, (b, kv-head) crossings
+    (1, 700, 16, 1, 64, 1.0, True),    # scores grow along the sequence: running max moves often
+    (1, 2049, 8, 1, 16, 1.0, True),
+])
+def test_ga_pair_kernel(cuda_device, B, n, hq, hkv, rot, k_scale, ramp):
+    """Full causal prefix with 8 or 16 query heads per KV head: the kernel that pairs two
+    row blocks per work item and rescales its output only when the running max jumps."""
+    inp = wl.prefill_inputs(B, n, hq, hkv, seed=250 + n + hq, k_scale=k_scale)
+    if ramp:
+        # A shared offset on the unrotated dims of q (+1) and k (+2 t / n) adds about
+        # 128 * 2 t / (n sqrt(192)) ~ 18 t / n to every score of key t, so the row max keeps
+        # climbing from tile to tile while the values stay small enough for f16 rounding.
+        shift = 2.0 * torch.arange(n, dtype=torch.float32) / n
+        k = inp["k"].float()
+        k[..., 64:] += shift[None, :, None, None]
+        q = inp["q"].float()
+        q[..., 64:] += 1.0
+        inp["k"], inp["q"] = k.to(torch.bfloat16), q.to(torch.bfloat16)
+    _run_and_compare(inp, 0, wl.GA_THETA, rot, cuda_device, f"ga-pair B={B} n={n} {hq}/{hkv}")
+
+
 def test_window_ge_n_equals_ga(cuda_device):
     """W >= n is full causal attention: same result as window = 0, bit for bit."""
     inp = wl.prefill_inputs(1, 200, 8, 1, seed=7)
