@@ -493,7 +493,7 @@ def main():
                 "workload": wl.GA_PREFILL.name, "value": round(ga["flops"] / (ms_ga * 1e-3) / 1e12, 2),
                 "unit": "TFLOP/s", "ms_per_step": round(ms_ga, 4),
                 "roofline": roofline_tensor(ga["flops"], ms_ga, peaks["bf16_tflops"], tag,
-                                            traffic_for("prefill_kernel_ga", wl.GA_PREFILL.seqlen)),
+                                            traffic_for("prefill_ga_kernel", wl.GA_PREFILL.seqlen)),
                 "device_error": ga["device_error"]}
             del ga
             torch.cuda.empty_cache()

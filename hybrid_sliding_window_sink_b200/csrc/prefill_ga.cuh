@@ -24,10 +24,44 @@
 // reference moves.
 #pragma once
 
+#include <type_traits>
+
 #include "ptx.cuh"
 #include "prefill.cuh"
 
 namespace mimo {
+
+// max of three floats in one instruction (sm_100 three-input max).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Two floats -> packed f16x2, round to nearest even, saturating to the finite f16 range.
+__device__ __forceinline__ uint32_t pack_f16_satfinite(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// 32 consecutive TMEM columns of this warp's 32 lanes.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  tmem_ld16(taddr, *reinterpret_cast<uint32_t(*)[16]>(r));
+  tmem_ld16(taddr + 16, *reinterpret_cast<uint32_t(*)[16]>(r + 16));
+}
+// Placed right after tmem_wait_ld(): makes every later use of r depend on this point, so
+// the compiler cannot move arithmetic on TMEM-loaded registers above the wait.
+__device__ __forceinline__ void reg_fence16(uint32_t (&r)[16]) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                 "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]),
+                 "+r"(r[13]), "+r"(r[14]), "+r"(r[15]));
+}
+__device__ __forceinline__ void reg_fence32(uint32_t (&r)[32]) {
+  reg_fence16(*reinterpret_cast<uint32_t(*)[16]>(r));
+  reg_fence16(*reinterpret_cast<uint32_t(*)[16]>(r + 16));
+}
 
 constexpr int kGaThreads = 448;
 constexpr int kGaBN = 128;
@@ -155,19 +189,25 @@ __global__ void __launch_bounds__(kGaThreads, 1)
             tma_load_4d(sQ + blk * L::Q_BLOCK + c * L::Q_CHUNK, &tmQ, bar(kGaQFull), 64 * c, g * G,
                         p0 + blk * P, b);
         ++nq;
-        for (int j = 0; j < T; ++j) {
-          const int ks = nk & 1;
-          if (nk >= 2 && !mbar_wait(bar(kGaKEmpty + ks), ((nk >> 1) - 1) & 1, s_abort, err)) { ok = false; break; }
-          mbar_arrive_expect_tx(bar(kGaKFull + ks), L::K_TILE);
-          for (int c = 0; c < 3; ++c)
-            tma_load_4d(sK + ks * L::K_TILE + c * L::K_CHUNK, &tmK, bar(kGaKFull + ks), 64 * c, g,
-                        j * kGaBN, b);
-          ++nk;
-          if (nv >= 1 && !mbar_wait(bar(kGaVEmpty), (nv - 1) & 1, s_abort, err)) { ok = false; break; }
-          mbar_arrive_expect_tx(bar(kGaVFull), L::V_TILE);
-          for (int c = 0; c < 2; ++c)
-            tma_load_4d(sV + c * L::K_CHUNK, &tmV, bar(kGaVFull), 64 * c, g, j * kGaBN, b);
-          ++nv;
+        // K runs one tile ahead of V: K(j + 1) needs only S of tile j - 1 to be done,
+        // while the single V buffer frees up only when PV of tile j - 1 is done
+        for (int j = 0; j <= T && ok; ++j) {
+          if (j < T) {
+            const int ks = nk & 1;
+            if (nk >= 2 && !mbar_wait(bar(kGaKEmpty + ks), ((nk >> 1) - 1) & 1, s_abort, err)) { ok = false; break; }
+            mbar_arrive_expect_tx(bar(kGaKFull + ks), L::K_TILE);
+            for (int c = 0; c < 3; ++c)
+              tma_load_4d(sK + ks * L::K_TILE + c * L::K_CHUNK, &tmK, bar(kGaKFull + ks), 64 * c, g,
+                          j * kGaBN, b);
+            ++nk;
+          }
+          if (j >= 1) {
+            if (nv >= 1 && !mbar_wait(bar(kGaVEmpty), (nv - 1) & 1, s_abort, err)) { ok = false; break; }
+            mbar_arrive_expect_tx(bar(kGaVFull), L::V_TILE);
+            for (int c = 0; c < 2; ++c)
+              tma_load_4d(sV + c * L::K_CHUNK, &tmV, bar(kGaVFull), 64 * c, g, (j - 1) * kGaBN, b);
+            ++nv;
+          }
         }
       }
       if (!ok) {   // let every issued copy land before the CTA can exit
@@ -350,8 +390,8 @@ __global__ void __launch_bounds__(kGaThreads, 1)
                     r1[h] = x1 * c - x2 * sn;
                     r2[h] = x2 * c + x1 * sn;
                   }
-                  xs[e2] = pack_f16_sat(r1[0], r1[1]);
-                  ys[e2] = pack_f16_sat(r2[0], r2[1]);
+                  xs[e2] = pack_f16_satfinite(r1[0], r1[1]);
+                  ys[e2] = pack_f16_satfinite(r2[0], r2[1]);
                 }
                 *px = make_uint4(xs[0], xs[1], xs[2], xs[3]);
                 *py = make_uint4(ys[0], ys[1], ys[2], ys[3]);
@@ -392,30 +432,35 @@ __global__ void __launch_bounds__(kGaThreads, 1)
         tc_fence_after();
         const int kt0 = j * kGaBN;
         const bool full = kt0 + kGaBN - 1 <= pmin;   // every key of the tile is <= every row's pos
-        // pass 1: tile max of the valid keys
+        // pass 1: tile max of the valid keys, 64 columns per TMEM round trip
         float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll 1
-        for (int c = 0; c < kGaBN / 16; c += 2) {
-          uint32_t v0[16], v1[16];
-          tmem_ld16(trow + c * 16, v0);
-          tmem_ld16(trow + (c + 1) * 16, v1);
+        for (int c = 0; c < kGaBN; c += 64) {
+          uint32_t v[64];
+          tmem_ld32(trow + c, *reinterpret_cast<uint32_t(*)[32]>(v));
+          tmem_ld32(trow + c + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
           tmem_wait_ld();
+          reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(v));
+          reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(v + 32));
           if (full) {
 #pragma unroll
-            for (int e = 0; e < 16; e += 2) {
-              mx0 = fmaxf(mx0, fmaxf(__uint_as_float(v0[e]), __uint_as_float(v0[e + 1])));
-              mx1 = fmaxf(mx1, fmaxf(__uint_as_float(v1[e]), __uint_as_float(v1[e + 1])));
+            for (int e = 0; e < 64; e += 4) {
+              mx0 = fmax3(mx0, __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+              mx1 = fmax3(mx1, __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
             }
           } else {
+            const int lim = pos - kt0 - c;   // columns e <= lim are keys <= pos
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              if (kt0 + c * 16 + e <= pos) mx0 = fmaxf(mx0, __uint_as_float(v0[e]));
-              if (kt0 + c * 16 + 16 + e <= pos) mx1 = fmaxf(mx1, __uint_as_float(v1[e]));
+            for (int e = 0; e < 64; e += 2) {
+              if (e <= lim) mx0 = fmaxf(mx0, __uint_as_float(v[e]));
+              if (e + 1 <= lim) mx1 = fmaxf(mx1, __uint_as_float(v[e + 1]));
             }
           }
         }
         const float tmax = fmaxf(mx0, mx1) * p.scale_log2;
-        // lazy reference update: move only when the max grows by more than 8 (or at tile 0)
+        // Reference update: the first tile of a row moves it to the tile max (the dominant P
+        // is then exactly 1); later tiles move it only when their max is 2^8 above it, so
+        // P = 2^(a - ref) stays below 2^8 and O, l are rescaled only when the reference moves.
         const bool move = (j == 0) ? (tmax > m) : (tmax > m + 8.f);
         float alpha = 1.f;
         if (move) {
@@ -425,51 +470,54 @@ __global__ void __launch_bounds__(kGaThreads, 1)
         }
         if (j > 0 && __any_sync(0xffffffffu, move)) {   // rescale O rows (warp-collective)
 #pragma unroll 1
-          for (int c = 0; c < 8; c += 2) {
-            uint32_t v0[16], v1[16];
-            tmem_ld16(trow + 128 + c * 16, v0);
-            tmem_ld16(trow + 128 + (c + 1) * 16, v1);
+          for (int c = 0; c < 128; c += 32) {
+            uint32_t v[32];
+            tmem_ld32(trow + 128 + c, v);
             tmem_wait_ld();
+            reg_fence32(v);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              v0[e] = __float_as_uint(__uint_as_float(v0[e]) * alpha);
-              v1[e] = __float_as_uint(__uint_as_float(v1[e]) * alpha);
-            }
-            tmem_st16(trow + 128 + c * 16, v0);
-            tmem_st16(trow + 128 + (c + 1) * 16, v1);
+            for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
+            tmem_st16(trow + 128 + c, *reinterpret_cast<const uint32_t(*)[16]>(v));
+            tmem_st16(trow + 128 + c + 16, *reinterpret_cast<const uint32_t(*)[16]>(v + 16));
           }
         }
         const float ref = m == -INFINITY ? 0.f : m;
         // pass 2: P = 2^(a - ref) (0 above the diagonal), bf16 into S columns [0, 64)
         float sa = 0.f, sb = 0.f;
+        auto pass2 = [&](auto masked) {
 #pragma unroll 1
-        for (int c = 0; c < kGaBN / 16; c += 2) {
-          uint32_t v0[16], v1[16];
-          tmem_ld16(trow + c * 16, v0);
-          tmem_ld16(trow + (c + 1) * 16, v1);
-          tmem_wait_ld();
-          uint32_t pk0[8], pk1[8];
+          for (int c = 0; c < kGaBN; c += 64) {
+            uint32_t v[64];
+            tmem_ld32(trow + c, *reinterpret_cast<uint32_t(*)[32]>(v));
+            tmem_ld32(trow + c + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+            tmem_wait_ld();
+            reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(v));
+            reg_fence32(*reinterpret_cast<uint32_t(*)[32]>(v + 32));
+            const int lim = pos - kt0 - c;   // columns e <= lim are keys <= pos
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            float a0 = ex2(fmaf(__uint_as_float(v0[2 * e]), p.scale_log2, -ref));
-            float a1 = ex2(fmaf(__uint_as_float(v0[2 * e + 1]), p.scale_log2, -ref));
-            float b0 = ex2(fmaf(__uint_as_float(v1[2 * e]), p.scale_log2, -ref));
-            float b1 = ex2(fmaf(__uint_as_float(v1[2 * e + 1]), p.scale_log2, -ref));
-            if (!full) {
-              const int k0 = kt0 + c * 16 + 2 * e;
-              a0 = k0 <= pos ? a0 : 0.f;
-              a1 = k0 + 1 <= pos ? a1 : 0.f;
-              b0 = k0 + 16 <= pos ? b0 : 0.f;
-              b1 = k0 + 17 <= pos ? b1 : 0.f;
+            for (int q = 0; q < 4; ++q) {
+              uint32_t pk[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const int col = 16 * q + 2 * e;
+                float a0 = ex2(fmaf(__uint_as_float(v[col]), p.scale_log2, -ref));
+                float a1 = ex2(fmaf(__uint_as_float(v[col + 1]), p.scale_log2, -ref));
+                if (decltype(masked)::value) {
+                  a0 = col <= lim ? a0 : 0.f;
+                  a1 = col + 1 <= lim ? a1 : 0.f;
+                }
+                sa += a0;
+                sb += a1;
+                pk[e] = pack_bf16(a0, a1);
+              }
+              tmem_st8(trow + (c >> 1) + 8 * q, pk);
             }
-            sa += a0 + a1;
-            sb += b0 + b1;
-            pk0[e] = pack_bf16(a0, a1);
-            pk1[e] = pack_bf16(b0, b1);
           }
-          tmem_st8(trow + c * 8, pk0);
-          tmem_st8(trow + (c + 1) * 8, pk1);
-        }
+        };
+        if (full)
+          pass2(std::false_type{});
+        else
+          pass2(std::true_type{});
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(kGaPReady + grp));
