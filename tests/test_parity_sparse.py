@@ -42,6 +42,28 @@ def test_sparse_small(cuda_device, B, hq, hkv, cap, lengths, recent, n_sel):
     compare(wl.to_f64(out), o_ref, wl.to_f64(lse), l_ref, f"sparse {lengths}")
 
 
+@pytest.mark.parametrize("B,hq,hkv,n_sel", [
+    (15, 64, 4, 300),     # 60 (b, g) units of 428 keys, 16 heads per KV head
+    (40, 32, 4, 100),     # 160 units, 8 heads per KV head
+    (80, 16, 4, 64),      # 320 units (more than two per SM), 4 heads per KV head
+])
+def test_sparse_many_units(cuda_device, B, hq, hkv, n_sel):
+    """Sparse calls over many (b, g) units with ragged lengths per sequence (different
+    chunk plans and group sizes)."""
+    r = np.random.default_rng(B + n_sel)
+    cap = 512
+    recent = 128
+    lengths = [int(x) for x in r.integers(recent + n_sel, cap + 1, size=B)]
+    inp = _inputs(B, hq, hkv, cap, lengths, recent, n_sel, seed=500 + B)
+    out, lse = _run(inp, recent, cuda_device)
+    torch.cuda.synchronize()
+    assert _lib.last_device_error() == 0
+    o_ref, l_ref = ref.sparse_decode(wl.to_f64(inp["q"]), wl.to_f64(inp["k_cache"]),
+                                     wl.to_f64(inp["v_cache"]), lengths, recent,
+                                     inp["sel"].numpy(), wl.to_f64(inp["sink"]))
+    compare(wl.to_f64(out), o_ref, wl.to_f64(lse), l_ref, f"sparse B={B} n_sel={n_sel}")
+
+
 def test_sparse_full_config(cuda_device):
     """B=8, L=262144, 64/4, recent 128 + 1,024 sorted unique indices: every output."""
     c = wl.SPARSE_DECODE
