@@ -22,6 +22,10 @@ Sources (page title and section):
 * "小米MiMo-V3的核心架构HySparse2" (aideepthink.cn): §二.2 / §四.3 token-level
   selection, most recent 128 tokens plus 1,024 selected tokens in one merged
   sparse attention over one shared KV cache.
+* syt-nju.github.io visual reading "mimo-mtp-swa-not-mla", MTP section: three draft
+  tokens verified in one forward pass of the main model (speculative decoding).
+* youngju.dev "mimo-v25-inference-optimization", KV-cache section: a dual pool, the
+  SWA pool holding O(W) slots per sequence.
 
 Readings where the pages are silent (each also listed in the design notes):
 
@@ -34,6 +38,9 @@ Readings where the pages are silent (each also listed in the design notes):
   (d, d + rot_dims/2) and inverse frequency theta**(-2k/rot_dims).
 * GQA: query head h reads KV head h // (Hq // Hkv).
 * Ring cache: token p of a sequence lives in slot p mod capacity.
+* Multi-query decode: the T newest tokens of a sequence (positions L-T .. L-1, all
+  already written to the cache) are verified together; each has its own window
+  (SWA) or causal prefix (GA), exactly as the same rows of a prefill would.
 """
 
 from __future__ import annotations
@@ -51,6 +58,7 @@ __all__ = [
     "prefill",
     "prefill_rows",
     "decode",
+    "decode_multi",
     "sparse_decode",
     "sparse_key_set",
     "partial_state",
@@ -281,6 +289,49 @@ def decode(q, k_cache, v_cache, kind: str, lengths, sink, scale=None):
             g = h // group
             o[b, h], lse[b, h] = attend_row(q[b, h], kc[b, :, g, :], vc[b, :, g, :], slots,
                                             None if sink is None else float(sink[h]), sc)
+    return o, lse
+
+
+def _multi_rows(kind: str, L: int, T: int, t: int, capacity: int, window: int) -> np.ndarray:
+    """Cache slots draft token t (position p = L - T + t) attends in multi-query decode.
+
+    ring: the tokens of its window [max(0, p-W+1), p], at slots token mod capacity; the
+    ring must still hold all of them (capacity >= W + T - 1 covers every t); linear:
+    tokens 0..p at slots 0..p.
+    """
+    if not 1 <= T <= L:
+        raise ValueError("multi-query decode needs 1 <= T <= L")
+    p = L - T + t
+    if kind == "ring":
+        lo = max(0, p - window + 1)
+        if lo < L - capacity:
+            raise ValueError("ring too small: part of the window was overwritten")
+        return np.arange(lo, p + 1, dtype=np.int64) % capacity
+    if kind == "linear":
+        if L > capacity:
+            raise ValueError("length exceeds linear cache capacity")
+        return np.arange(p + 1, dtype=np.int64)
+    raise ValueError(kind)
+
+
+def decode_multi(q, k_cache, v_cache, kind: str, lengths, window: int, sink, scale=None):
+    """Multi-query decode (MTP draft verification). q: [B, T, Hq, Dqk], the already
+    rotated queries of the T newest tokens of each sequence; caches as in decode().
+    Returns (o [B, T, Hq, Dv], lse [B, T, Hq])."""
+    q, kc, vc = _f64(q), _f64(k_cache), _f64(v_cache)
+    B, T, Hq, D = q.shape
+    cap, Hkv = kc.shape[1], kc.shape[2]
+    group = Hq // Hkv
+    sc = _scale(scale, D)
+    o = np.zeros((B, T, Hq, vc.shape[-1]))
+    lse = np.zeros((B, T, Hq))
+    for b in range(B):
+        for t in range(T):
+            slots = _multi_rows(kind, int(lengths[b]), T, t, cap, window)
+            for h in range(Hq):
+                g = h // group
+                o[b, t, h], lse[b, t, h] = attend_row(q[b, t, h], kc[b, :, g, :], vc[b, :, g, :],
+                                                      slots, None if sink is None else float(sink[h]), sc)
     return o, lse
 
 

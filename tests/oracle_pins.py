@@ -303,6 +303,47 @@ def check_decode_matches_prefill(ref):
         np.testing.assert_allclose(lse2[0], lse_ga[0, :, L - 1], rtol=0, atol=1e-11)
 
 
+def check_multi_decode_matches_prefill(ref):
+    """MTP verification (syt-nju "mimo-mtp-swa-not-mla", MTP section): the T newest
+    tokens of a sequence, verified together against the cache, give the last T rows of
+    a prefill of the same sequence: on a ring of capacity >= W + T - 1 (token p in slot
+    p mod capacity, with wrap-around) for SWA, on a linear cache for GA. T = 1 is the
+    one-token decode. A ring that has lost part of a draft token's window is refused."""
+    n, hq, hkv, d, dv, W = 90, 4, 2, 16, 8, 12
+    q, k, v, sink = _rand_prefill(23, n=n, hq=hq, hkv=hkv, d=d, dv=dv)
+    for T, cap in ((1, 12), (3, 14), (4, 16), (4, 21)):
+        for L in (T, T + 1, W, W + T, 40, 90):
+            if L < T or L > n:
+                continue
+            pos = np.arange(L, dtype=np.float64)
+            kr = ref.rope(k[0, :L], pos, 1e4, 8)
+            qr = ref.rope(q[0, L - T:L], pos[L - T:], 1e4, 8)
+            o_pf, lse_pf = ref.prefill(q[:, :L], k[:, :L], v[:, :L], sink, W, 1e4, 8)
+            ring_k = np.zeros((1, cap, hkv, d))
+            ring_v = np.zeros((1, cap, hkv, dv))
+            for p in range(L):
+                ring_k[0, p % cap] = kr[p]
+                ring_v[0, p % cap] = v[0, p]
+            o, lse = ref.decode_multi(qr[None], ring_k, ring_v, "ring", [L], W, sink)
+            np.testing.assert_allclose(o[0], o_pf[0, L - T:L], rtol=1e-11, atol=1e-12)
+            np.testing.assert_allclose(lse[0], lse_pf[0, :, L - T:L].T, rtol=0, atol=1e-11)
+            o_ga, lse_ga = ref.prefill(q[:, :L], k[:, :L], v[:, :L], sink, 0, 1e4, 8)
+            o2, lse2 = ref.decode_multi(qr[None], kr[None], v[:, :L], "linear", [L], 0, sink)
+            np.testing.assert_allclose(o2[0], o_ga[0, L - T:L], rtol=1e-11, atol=1e-12)
+            np.testing.assert_allclose(lse2[0], lse_ga[0, :, L - T:L].T, rtol=0, atol=1e-11)
+            if T == 1:
+                o1, l1 = ref.decode(qr, ring_k, ring_v, "ring", [L], sink)
+                np.testing.assert_allclose(o[0, 0], o1[0], rtol=1e-13, atol=1e-14)
+                np.testing.assert_allclose(lse[0, 0], l1[0], rtol=0, atol=1e-13)
+    try:
+        ring = np.zeros((1, W + 1, hkv, d))
+        ref.decode_multi(q[:, :3], ring, ring[..., :dv], "ring", [40], W, sink)
+    except ValueError:
+        pass
+    else:
+        raise AssertionError("a ring without room for every draft token's window must be refused")
+
+
 def check_sparse_membership(ref):
     """aideepthink.cn §四.3: the key set is the most recent ``recent`` tokens
     plus the selected ones, in one softmax. One-hot values expose membership."""
@@ -380,6 +421,7 @@ ALL_CHECKS = [
     check_rope_relative,
     check_split_combine,
     check_decode_matches_prefill,
+    check_multi_decode_matches_prefill,
     check_sparse_membership,
     check_golden,
 ]

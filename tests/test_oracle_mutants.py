@@ -36,6 +36,12 @@ MUTANTS = {
     "combine counts sink per chunk": ("L += math.exp(float(sink) - M)", "L += len(parts) * math.exp(float(sink) - M)"),
     "combine without rescale": ("o = sum(oc * math.exp(m - M) for m, _, oc in parts) / L",
                                 "o = sum(oc for m, _, oc in parts) / L"),
+    "draft tokens all at the last position": ("    p = L - T + t\n", "    p = L - 1\n"),
+    "draft window one too wide": ("lo = max(0, p - window + 1)", "lo = max(0, p - window)"),
+    "draft ring slot without modulo": ("return np.arange(lo, p + 1, dtype=np.int64) % capacity",
+                                       "return np.arange(lo, p + 1, dtype=np.int64) - max(0, L - capacity)"),
+    "draft causal prefix excludes itself": ("        return np.arange(p + 1, dtype=np.int64)\n",
+                                            "        return np.arange(p, dtype=np.int64)\n"),
 }
 
 
