@@ -26,7 +26,7 @@ STATUS = {0: "MIMO_OK", 1: "MIMO_ERR_NULL", 2: "MIMO_ERR_SHAPE", 3: "MIMO_ERR_UN
 
 #: Every symbol include/mimo_attn.h declares.
 EXPORTS = ("mimo_attn_prefill", "mimo_attn_decode", "mimo_attn_sparse", "mimo_attn_sparse_noalloc",
-           "mimo_attn_workspace_size",
+           "mimo_attn_decode_mq", "mimo_attn_decode_mq_workspace_size", "mimo_attn_workspace_size",
            "mimo_attn_check_indices", "mimo_attn_last_device_error", "mimo_status_string",
            "mimo_attn_version")
 
@@ -64,6 +64,9 @@ def lib():
     L.mimo_attn_decode.argtypes = [SP, P, P, P, I, I, LL, P, P, P, P, P, SZ, P]
     L.mimo_attn_sparse.argtypes = [SP, P, P, P, I, LL, P, I, P, I, P, P, P, P, SZ, P]
     L.mimo_attn_sparse_noalloc.argtypes = [SP, P, P, P, I, LL, P, I, P, I, P, P, P, P]
+    L.mimo_attn_decode_mq.argtypes = [SP, P, P, P, I, I, LL, P, I, I, P, P, P, P, SZ, P]
+    L.mimo_attn_decode_mq_workspace_size.argtypes = [SP, I, I, I, I]
+    L.mimo_attn_decode_mq_workspace_size.restype = SZ
     L.mimo_attn_workspace_size.argtypes = [SP, I, I, I, I, I]
     L.mimo_attn_workspace_size.restype = SZ
     L.mimo_attn_check_indices.argtypes = [SP, P, P, I, I, I, P, P]
@@ -186,6 +189,38 @@ def decode(q, k_cache, v_cache, lengths, sink=None, *, kind="ring", capacity=Non
                                 cap, stride, _ptr(lengths), _ptr(sink), _ptr(out), _ptr(lse),
                                 _ptr(ws), nbytes, _stream(stream))
     _check("mimo_attn_decode", st)
+    return out, lse
+
+
+def decode_mq(q, k_cache, v_cache, lengths, sink=None, *, kind="ring", window=128, capacity=None,
+              softmax_scale=0.0, out=None, lse=None, want_lse=True, workspace=None, stream=None):
+    """mimo_attn_decode_mq. q [B,T,Hq,192] (the T newest tokens of each sequence, rotated);
+    caches [B,stride,Hkv,192/128] bf16 holding them; lengths [B] int32 including them.
+    kind "ring" (slot p mod capacity, needs capacity >= window + T - 1) or "linear"."""
+    _need(q, "q", torch.bfloat16, 4)
+    _need(k_cache, "k_cache", torch.bfloat16, 4)
+    _need(v_cache, "v_cache", torch.bfloat16, 4)
+    _need(lengths, "lengths", torch.int32, 1)
+    B, T, hq, dqk = q.shape
+    _, stride, hkv, _ = k_cache.shape
+    if v_cache.shape[:3] != (B, stride, hkv) or k_cache.shape[0] != B or lengths.shape[0] != B:
+        raise ValueError("cache / lengths shapes disagree with q")
+    cap = stride if capacity is None else int(capacity)
+    kind_id = {"ring": MIMO_CACHE_RING, "linear": MIMO_CACHE_LINEAR}[kind]
+    if sink is not None:
+        _need(sink, "sink", torch.float32, 1)
+    if out is None:
+        out = torch.empty(B, T, hq, v_cache.shape[3], dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty(B, T, hq, dtype=torch.float32, device=q.device)
+    shape = make_shape(B, 1, hq, hkv, dqk, v_cache.shape[3], softmax_scale)
+    nbytes = int(lib().mimo_attn_decode_mq_workspace_size(ctypes.byref(shape), kind_id, cap, T,
+                                                          int(window)))
+    ws = _workspace(workspace, nbytes, q.device)
+    st = lib().mimo_attn_decode_mq(ctypes.byref(shape), _ptr(q), _ptr(k_cache), _ptr(v_cache), kind_id,
+                                   cap, stride, _ptr(lengths), T, int(window), _ptr(sink), _ptr(out),
+                                   _ptr(lse), _ptr(ws), nbytes, _stream(stream))
+    _check("mimo_attn_decode_mq", st)
     return out, lse
 
 

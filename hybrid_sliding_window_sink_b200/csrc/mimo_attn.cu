@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -13,6 +14,7 @@
 #include "mimo_attn.h"
 #include "ptx.cuh"
 #include "decode.cuh"
+#include "decode_mq.cuh"
 #include "prefill.cuh"
 #include "prefill_swa.cuh"
 #include "prefill_ga.cuh"
@@ -334,6 +336,59 @@ mimo_status run_decode(const mimo_shape* s, int mode, const void* q, const void*
   }
 }
 
+// ---------------------------------------------------------------- multi-query decode
+DecodePlan plan_decode_mq(const mimo_shape* s, int mode, int cap, int T, int W, int sms) {
+  DecodePlan pl{};
+  const long long units = static_cast<long long>(s->batch) * s->n_kv_heads;
+  long long total = mode == mimo::kModeRing ? std::min<long long>(cap, static_cast<long long>(W) + T - 1) : cap;
+  if (total < 1) total = 1;
+  if (total <= 256) {
+    pl.chunk = static_cast<int>((total + 63) / 64 * 64);
+  } else {
+    const long long c = total * units / (16LL * sms);
+    const int ch = pow2_floor(c);
+    pl.chunk = ch < 256 ? 256 : (ch > 4096 ? 4096 : ch);
+  }
+  pl.nchunks = static_cast<int>((total + pl.chunk - 1) / pl.chunk);
+  pl.direct = pl.nchunks == 1;
+  if (!pl.direct) {
+    const size_t rows = static_cast<size_t>(s->batch) * T * s->n_q_heads * pl.nchunks;
+    const size_t ml = (rows * 2 * sizeof(float) + 255) / 256 * 256;
+    pl.bytes = ml + rows * mimo::kDV * sizeof(float);
+  }
+  return pl;
+}
+
+mimo_status check_mq(const mimo_shape* s, int cache_kind, int cap, int T, int W) {
+  mimo_status e = check_heads(s);
+  if (e != MIMO_OK) return e;
+  if (cache_kind != MIMO_CACHE_RING && cache_kind != MIMO_CACHE_LINEAR) return MIMO_ERR_SHAPE;
+  if (T < 1 || cap < 1) return MIMO_ERR_SHAPE;
+  if (static_cast<long long>(T) * (s->n_q_heads / s->n_kv_heads) > mimo::kMqMaxRows) return MIMO_ERR_UNSUPPORTED;
+  if (cache_kind == MIMO_CACHE_RING && (W < 1 || static_cast<long long>(W) + T - 1 > cap)) return MIMO_ERR_SHAPE;
+  return MIMO_OK;
+}
+
+template <int G>
+mimo_status launch_decode_mq_g(const mimo::DecodeMqParams& prm, cudaStream_t st) {
+  auto kern = mimo::decode_mq_kernel<G>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, mimo::kDecSmemBytes) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return MIMO_ERR_CUDA;
+  }
+  dim3 grid(prm.nchunks, prm.Hkv, prm.B);
+  kern<<<grid, mimo::kDecThreads, mimo::kDecSmemBytes, st>>>(prm);
+  if (cudaGetLastError() != cudaSuccess) return MIMO_ERR_CUDA;
+  if (!prm.direct) {
+    const long long rows = static_cast<long long>(prm.B) * prm.T * prm.Hq;
+    if (rows > 0x7fffffffLL) return MIMO_ERR_UNSUPPORTED;
+    mimo::decode_mq_combine_kernel<<<static_cast<unsigned>(rows), mimo::kDV, 0, st>>>(prm);
+    if (cudaGetLastError() != cudaSuccess) return MIMO_ERR_CUDA;
+  }
+  return MIMO_OK;
+}
+
 }  // namespace
 
 // ============================================================== C ABI
@@ -401,6 +456,70 @@ mimo_status mimo_attn_sparse(const mimo_shape* s, const void* q, const void* k_c
   return run_decode(s, mimo::kModeSparse, q, k_cache, v_cache, cache_capacity, seq_stride_tokens,
                     lengths, recent, sel_idx, n_sel, sink, out, lse, workspace, workspace_bytes,
                     stream);
+}
+
+mimo_status mimo_attn_decode_mq(const mimo_shape* s, const void* q, const void* k_cache,
+                                const void* v_cache, int cache_kind, int cache_capacity,
+                                long long seq_stride_tokens, const int* lengths, int q_len,
+                                int window, const float* sink, void* out, float* lse,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+  mimo_status e = check_mq(s, cache_kind, cache_capacity, q_len, window);
+  if (e != MIMO_OK) return e;
+  if (!q || !k_cache || !v_cache || !lengths || !out) return MIMO_ERR_NULL;
+  if (seq_stride_tokens < cache_capacity) return MIMO_ERR_SHAPE;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
+      !aligned(lengths, 4) || (sink && !aligned(sink, 4)) || (lse && !aligned(lse, 4)))
+    return MIMO_ERR_ALIGN;
+  const int dev = current_device();
+  if (dev < 0) return MIMO_ERR_CUDA;
+  const int mode = cache_kind == MIMO_CACHE_RING ? mimo::kModeRing : mimo::kModeLinear;
+  const DecodePlan pl = plan_decode_mq(s, mode, cache_capacity, q_len, window, sm_count_for(dev));
+  if (pl.bytes > 0 && (!workspace || workspace_bytes < pl.bytes)) return MIMO_ERR_WORKSPACE;
+  if (workspace && !aligned(workspace, 16)) return MIMO_ERR_ALIGN;
+  if (s->n_kv_heads > 65535) return MIMO_ERR_UNSUPPORTED;
+  mimo::DecodeMqParams prm{};
+  prm.q = static_cast<const __nv_bfloat16*>(q);
+  prm.k = static_cast<const __nv_bfloat16*>(k_cache);
+  prm.v = static_cast<const __nv_bfloat16*>(v_cache);
+  prm.lengths = lengths;
+  prm.sink = sink;
+  prm.out = static_cast<__nv_bfloat16*>(out);
+  prm.lse = lse;
+  if (pl.bytes > 0) {
+    const size_t rows = static_cast<size_t>(s->batch) * q_len * s->n_q_heads * pl.nchunks;
+    const size_t ml = (rows * 2 * sizeof(float) + 255) / 256 * 256;
+    prm.part_ml = static_cast<float*>(workspace);
+    prm.part_o = reinterpret_cast<float*>(static_cast<char*>(workspace) + ml);
+  }
+  prm.seq_stride = seq_stride_tokens;
+  prm.B = s->batch;
+  prm.T = q_len;
+  prm.Hq = s->n_q_heads;
+  prm.Hkv = s->n_kv_heads;
+  prm.cap = cache_capacity;
+  prm.mode = mode;
+  prm.window = window;
+  prm.chunk = pl.chunk;
+  prm.nchunks = pl.nchunks;
+  prm.direct = pl.direct;
+  prm.scale_log2 = scale_log2_of(s);
+  prm.err = device_error_ptr(dev);
+  if (!prm.err) return MIMO_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  switch (s->n_q_heads / s->n_kv_heads) {
+    case 1: return launch_decode_mq_g<1>(prm, st);
+    case 2: return launch_decode_mq_g<2>(prm, st);
+    case 4: return launch_decode_mq_g<4>(prm, st);
+    case 8: return launch_decode_mq_g<8>(prm, st);
+    default: return launch_decode_mq_g<16>(prm, st);
+  }
+}
+
+size_t mimo_attn_decode_mq_workspace_size(const mimo_shape* s, int cache_kind, int cache_capacity,
+                                          int q_len, int window) {
+  if (check_mq(s, cache_kind, cache_capacity, q_len, window) != MIMO_OK) return 0;
+  const int mode = cache_kind == MIMO_CACHE_RING ? mimo::kModeRing : mimo::kModeLinear;
+  return plan_decode_mq(s, mode, cache_capacity, q_len, window, sm_count_for(current_device())).bytes;
 }
 
 size_t mimo_attn_workspace_size(const mimo_shape* s, int op, int cache_kind, int cache_capacity,

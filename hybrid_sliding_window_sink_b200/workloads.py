@@ -141,6 +141,16 @@ def decode_inputs(batch, hq, hkv, capacity, lengths, *, seed, device="cpu",
             "lengths": torch.as_tensor(lengths, dtype=torch.int32).to(device)}
 
 
+def decode_mq_inputs(batch, q_len, hq, hkv, capacity, lengths, *, seed, device="cpu",
+                     dqk=DQK, dv=DV):
+    """Multi-query decode inputs: those of decode_inputs (same draws) plus
+    ``q_mq`` [B, q_len, Hq, dqk] bf16 for the q_len newest tokens, drawn after them."""
+    inp = decode_inputs(batch, hq, hkv, capacity, lengths, seed=seed, device=device, dqk=dqk, dv=dv)
+    g = _gen(seed + 29, device)
+    inp["q_mq"] = _randn_bf16((batch, q_len, hq, dqk), g, device)
+    return inp
+
+
 def sorted_unique_indices(batch, hkv, n_sel, hi_excl, *, seed):
     """[B, Hkv, n_sel] int32, each row sorted unique uniform in [0, hi_excl[b])."""
     g = _gen(seed + 13, "cpu")

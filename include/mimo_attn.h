@@ -152,6 +152,46 @@ mimo_status mimo_attn_sparse(const mimo_shape* shape, const void* q, const void*
                              float* lse, void* workspace, size_t workspace_bytes,
                              void* stream);
 
+/*
+ * Multi-query decode: MTP draft verification (syt-nju.github.io "mimo-mtp-swa-not-mla",
+ * MTP section: the main model checks the draft tokens in one forward pass). The q_len
+ * newest tokens of each sequence, at positions L_b - q_len .. L_b - 1 and already written
+ * to the cache, are attended together; draft token t (position p = L_b - q_len + t) sees
+ *   MIMO_CACHE_RING   (SWA pool; token p in slot p mod cache_capacity): tokens
+ *                     [max(0, p - window + 1), p]; needs cache_capacity >= window + q_len - 1
+ *                     so that no draft token's window has been overwritten;
+ *   MIMO_CACHE_LINEAR (GA pool): tokens [0, p] (window ignored).
+ * With q_len = 1 on a ring of window slots this is mimo_attn_decode.
+ *
+ *  shape            batch, n_q_heads, n_kv_heads, head dims (192 / 128), softmax_scale;
+ *                   seqlen is ignored
+ *  q       [B, q_len, Hq, 192] bf16 device, already rotated, contiguous
+ *  k_cache, v_cache, cache_kind, cache_capacity, seq_stride_tokens, sink: as in
+ *                   mimo_attn_decode (K stored rotated)
+ *  lengths [B] int32 device: tokens in the cache per sequence including the draft tokens;
+ *                   precondition q_len <= L_b (draft tokens before position 0 have no keys)
+ *  q_len            draft tokens per sequence, 1 <= q_len and q_len * Hq/Hkv <= 64
+ *  window           SWA window W >= 1 (ring only)
+ *  out     [B, q_len, Hq, 128] bf16 device; lse [B, q_len, Hq] fp32 device or NULL
+ *  workspace        at least mimo_attn_decode_mq_workspace_size(...) bytes (may be NULL
+ *                   when that is 0)
+ *
+ * Each (sequence, KV head) unit reads its key range [min_t window start, L_b) once for all
+ * q_len * Hq/Hkv query rows. Errors as mimo_attn_decode; MIMO_ERR_SHAPE also when the ring
+ * is smaller than window + q_len - 1 or window < 1; MIMO_ERR_UNSUPPORTED when
+ * q_len * Hq/Hkv > 64.
+ */
+mimo_status mimo_attn_decode_mq(const mimo_shape* shape, const void* q, const void* k_cache,
+                                const void* v_cache, int cache_kind, int cache_capacity,
+                                long long seq_stride_tokens, const int* lengths, int q_len,
+                                int window, const float* sink, void* out, float* lse,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of device workspace mimo_attn_decode_mq needs for these sizes on the current device
+ * (0 when none is needed or the arguments are invalid). */
+size_t mimo_attn_decode_mq_workspace_size(const mimo_shape* shape, int cache_kind,
+                                          int cache_capacity, int q_len, int window);
+
 /* Bytes of device workspace mimo_attn_decode / mimo_attn_sparse need for these sizes
  * on the current device (0 when none is needed). Returns 0 for invalid arguments. */
 size_t mimo_attn_workspace_size(const mimo_shape* shape, int op, int cache_kind,

@@ -120,3 +120,40 @@ def test_workspace_size_plans(L):
     assert nsp > 0
     assert _lib.workspace_size(8, 64, 4, op=7, capacity=10) == 0
     assert _lib.workspace_size(8, 64, 4, op=_lib.MIMO_OP_SPARSE, capacity=10, recent=-1) == 0
+
+
+def _decode_mq(L, shape, kind=_lib.MIMO_CACHE_RING, cap=131, stride=131, q_len=4, window=128,
+               q=GOOD, k=GOOD, v=GOOD, lengths=GOOD, out=GOOD):
+    return L.mimo_attn_decode_mq(ctypes.byref(shape), q, k, v, kind, cap, stride, lengths, q_len,
+                                 window, None, out, None, None, 0, None)
+
+
+def test_decode_mq_rejects_before_launch(L):
+    s16 = _shape(hq=64, hkv=4)                       # 16 query heads per KV head
+    # ring must keep every draft token's window: capacity >= window + q_len - 1
+    assert _decode_mq(L, s16, cap=130, stride=130) == 2
+    assert _decode_mq(L, s16, window=0) == 2
+    assert _decode_mq(L, s16, q_len=0) == 2
+    assert _decode_mq(L, s16, kind=7) == 2
+    assert _decode_mq(L, s16, q_len=5) == 3          # 5 * 16 rows > 64
+    assert _decode_mq(L, s16, q=None) == 1
+    assert _decode_mq(L, s16, stride=100) == 2       # stride below capacity
+    assert _decode_mq(L, s16, q=P(0x10002)) == 4     # misaligned
+    # linear cache ignores the window
+    assert _decode_mq(L, s16, kind=_lib.MIMO_CACHE_LINEAR, window=0, cap=4096, stride=4096,
+                      q=None) == 1
+
+
+def test_decode_mq_workspace_plans(L):
+    ring = _shape(batch=64, hq=64, hkv=8)
+    # a ring of window + 3 slots fits one chunk: finalised in place
+    assert L.mimo_attn_decode_mq_workspace_size(ctypes.byref(ring), _lib.MIMO_CACHE_RING, 131, 4,
+                                                128) == 0
+    lin = _shape(batch=64, hq=64, hkv=4)
+    n = L.mimo_attn_decode_mq_workspace_size(ctypes.byref(lin), _lib.MIMO_CACHE_LINEAR, 131072, 4, 0)
+    assert n > 0 and n % 4 == 0
+    # invalid sizes: no plan
+    assert L.mimo_attn_decode_mq_workspace_size(ctypes.byref(ring), _lib.MIMO_CACHE_RING, 128, 4,
+                                                128) == 0
+    assert L.mimo_attn_decode_mq_workspace_size(ctypes.byref(lin), _lib.MIMO_CACHE_LINEAR, 4096, 8,
+                                                0) == 0
