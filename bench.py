@@ -17,6 +17,7 @@ job time is the max over ranks.
 from __future__ import annotations
 
 import argparse
+import ctypes
 import json
 import os
 import statistics
@@ -335,6 +336,80 @@ def bench_decode_step(steps, warmup, peaks, tag, dev, stream):
     return res
 
 
+def mtp_layer_bytes(lengths, hq, hkv, kind, cap, q_len):
+    """Algorithmic bytes of one multi-query decode layer: each (sequence, KV head) reads its
+    key range once (ring: min(L, cap) <= W + q_len - 1 tokens; linear: L tokens), plus q,
+    out and lse of the q_len rows per query head."""
+    L = np.asarray(lengths, dtype=np.int64)
+    keys = np.minimum(L, cap) if kind == "ring" else L
+    kv = int(keys.sum()) * hkv * (wl.DQK + wl.DV) * 2
+    rows = len(L) * q_len * hq
+    return float(kv + rows * (wl.DQK * 2 + wl.DV * 2 + 4) + hq * 4 + len(L) * 4)
+
+
+def bench_mtp_step(steps, warmup, peaks, tag, dev, stream, q_len=4):
+    """MTP verification step over the 48-layer hybrid pattern (B=64, 1 + 3 draft tokens per
+    sequence): 39 SWA layers on distinct rings of W + q_len - 1 = 131 slots, 9 GA layers on one
+    padded linear cache (131072 slots). Lengths as the decode step."""
+    from hybrid_sliding_window_sink_b200 import _lib
+    cs, cg = wl.HYBRID_DECODE_SWA, wl.HYBRID_DECODE_GA
+    cap_ring = wl.SWA_WINDOW + q_len - 1
+    L = wl.lengths_uniform(cs.batch, cs.min_len, cs.max_len, seed=cs.seed)
+    Ld = L.to(dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(cs.seed + 5)
+    layers = []
+    ga_k = torch.randn(cg.batch, cg.capacity, cg.hkv, wl.DQK, generator=g, device=dev,
+                       dtype=torch.float32).to(torch.bfloat16)
+    ga_v = torch.randn(cg.batch, cg.capacity, cg.hkv, wl.DV, generator=g, device=dev,
+                       dtype=torch.float32).to(torch.bfloat16)
+    for kind in wl.layer_pattern():
+        hkv = cs.hkv if kind == 1 else cg.hkv
+        q = torch.randn(cs.batch, q_len, cs.hq, wl.DQK, generator=g, device=dev).to(torch.bfloat16)
+        sink = torch.randn(cs.hq, generator=g, device=dev)
+        if kind == 1:
+            kc = torch.randn(cs.batch, cap_ring, hkv, wl.DQK, generator=g, device=dev).to(torch.bfloat16)
+            vc = torch.randn(cs.batch, cap_ring, hkv, wl.DV, generator=g, device=dev).to(torch.bfloat16)
+        else:
+            kc, vc = ga_k, ga_v
+        out = torch.empty(cs.batch, q_len, cs.hq, wl.DV, dtype=torch.bfloat16, device=dev)
+        lse = torch.empty(cs.batch, q_len, cs.hq, dtype=torch.float32, device=dev)
+        layers.append((kind, q, kc, vc, sink, out, lse))
+    shape_ga = _lib.make_shape(cg.batch, 1, cg.hq, cg.hkv)
+    nws = int(_lib.lib().mimo_attn_decode_mq_workspace_size(ctypes.byref(shape_ga), _lib.MIMO_CACHE_LINEAR,
+                                                            cg.capacity, q_len, 0))
+    ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
+
+    def run_layer(lay):
+        kind, q, kc, vc, sink, out, lse = lay
+        _lib.decode_mq(q, kc, vc, Ld, sink, kind="ring" if kind == 1 else "linear",
+                       window=wl.SWA_WINDOW, out=out, lse=lse, workspace=ws, stream=stream)
+
+    ms = timed(lambda: [run_layer(l) for l in layers], steps, warmup, stream)
+    Ls = L.tolist()
+    b_swa = mtp_layer_bytes(Ls, cs.hq, cs.hkv, "ring", cap_ring, q_len)
+    b_ga = mtp_layer_bytes(Ls, cg.hq, cg.hkv, "linear", cg.capacity, q_len)
+    total = 39 * b_swa + 9 * b_ga
+    ga_layers = [l for l in layers if l[0] == 0]
+    swa_layers = [l for l in layers if l[0] == 1]
+    ms_ga = timed(lambda: [run_layer(l) for l in ga_layers], steps, 1, stream) / (steps * 9)
+    ms_swa = timed(lambda: [run_layer(l) for l in swa_layers], steps, 1, stream) / (steps * 39)
+    flops_ga = 2.0 * (wl.DQK + wl.DV) * q_len * cg.hq * float(np.sum(Ls))   # upper bound: all keys
+    res = {
+        "value": round(total / (ms / steps * 1e-3) / 1e9, 1), "unit": "GB/s",
+        "ms_per_step": round(ms / steps, 4), "bytes_per_step": total, "q_len": q_len,
+        "launches_per_step": 39 + 9 * 2,
+        "ga_layer": roofline_hbm(b_ga, ms_ga, peaks, tag),
+        "swa_layer": roofline_hbm(b_swa, ms_swa, peaks, tag),
+        "roofline": roofline_hbm(total, ms / steps, peaks, tag),
+        "ms_ga_layer": round(ms_ga, 4), "ms_swa_layer": round(ms_swa, 5),
+        "ga_layer_tflops": round(flops_ga / (ms_ga * 1e-3) / 1e12, 1),
+        "cache": f"39 distinct SWA rings of {cap_ring} slots; one padded GA cache [64,131072,4,*]",
+    }
+    del layers, ga_k, ga_v, ws
+    return res
+
+
 def bench_sparse(steps, warmup, peaks, tag, dev, stream, calls=16):
     """Token-level sparse decode: ``calls`` independent calls (distinct q and index sets,
     >= 385 MB of gathered rows in all, more than L2) per step, captured in a CUDA graph."""
@@ -505,6 +580,12 @@ def main():
             torch.cuda.empty_cache()
         except Exception as e:
             wls["hybrid_decode_step"] = {"error": repr(e)}
+        try:
+            wls["mtp_decode_step"] = bench_mtp_step(max(3, ksteps), 3, peaks, tag, dev, stream)
+            wls["mtp_decode_step"]["workload"] = "MTP verification step (1+3 tokens), 48 layers, B=64"
+            torch.cuda.empty_cache()
+        except Exception as e:
+            wls["mtp_decode_step"] = {"error": repr(e)}
         try:
             wls["sparse_decode"] = bench_sparse(max(5, ksteps), 3, peaks, tag, dev, stream)
             wls["sparse_decode"]["workload"] = wl.SPARSE_DECODE.name

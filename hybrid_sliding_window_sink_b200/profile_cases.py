@@ -11,12 +11,15 @@ Cases:
   decode_ring_b256      SWA decode, B=256, ring of 128 slots, 64 Q / 8 KV heads
   decode_linear_b64_l16k GA decode, B=64, linear cache of 16384 tokens (all full), 64 Q / 4 KV heads
   sparse_b8_l65536      token-level sparse decode, B=8, L=65536, recent 128 + 1024 selected
+  mtp_linear_b64_l16k   multi-query (1 + 3 draft tokens) GA decode, B=64, linear cache of 16384
+                        tokens (all full), 64 Q / 4 KV heads
 Prints the mean time per call over --reps calls (after two warm-up calls).
 """
 
 from __future__ import annotations
 
 import argparse
+import ctypes
 import sys
 
 import torch
@@ -52,6 +55,14 @@ def _case(name, dev):
         sel = wl.sorted_unique_indices(8, 4, 1024, [L - 128] * 8, seed=9).to(dev)
         return lambda: _lib.sparse(d["q"], d["k_cache"], d["v_cache"], d["lengths"], sel, d["sink"],
                                    recent=128)
+    if name == "mtp_linear_b64_l16k":
+        d = wl.decode_mq_inputs(64, 4, 64, 4, 16384, [16384] * 64, seed=10, device=dev)
+        shape = _lib.make_shape(64, 1, 64, 4)
+        nws = int(_lib.lib().mimo_attn_decode_mq_workspace_size(ctypes.byref(shape),
+                                                               _lib.MIMO_CACHE_LINEAR, 16384, 4, 0))
+        ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
+        return lambda: _lib.decode_mq(d["q_mq"], d["k_cache"], d["v_cache"], d["lengths"], d["sink"],
+                                      kind="linear", window=0, workspace=ws)
     raise SystemExit(f"unknown case {name}")
 
 
