@@ -41,6 +41,10 @@ Readings where the pages are silent (each also listed in the design notes):
 * Multi-query decode: the T newest tokens of a sequence (positions L-T .. L-1, all
   already written to the cache) are verified together; each has its own window
   (SWA) or causal prefix (GA), exactly as the same rows of a prefill would.
+* FP8 KV cache (the pages size their KV caches in FP8 but give no scaling scheme):
+  K and V bytes are OCP FP8 E4M3 (bias 7, no infinities, S.1111.111 is NaN), each
+  (token, KV head) row carries one fp32 scale per tensor, and the cached value is
+  e4m3(byte) * scale. Attention then runs on those values exactly as on bf16 ones.
 """
 
 from __future__ import annotations
@@ -61,6 +65,10 @@ __all__ = [
     "decode_multi",
     "sparse_decode",
     "sparse_key_set",
+    "e4m3_to_float",
+    "dequant_fp8",
+    "decode_fp8",
+    "sparse_decode_fp8",
     "partial_state",
     "combine_partials",
 ]
@@ -398,3 +406,39 @@ def combine_partials(parts, sink):
         L += math.exp(float(sink) - M)
     o = sum(oc * math.exp(m - M) for m, _, oc in parts) / L
     return o, M + math.log(L)
+
+
+# --------------------------------------------------------------------------
+# FP8 (E4M3) KV cache
+# --------------------------------------------------------------------------
+
+def e4m3_to_float(bits) -> np.ndarray:
+    """Value of each OCP FP8 E4M3 byte: sign bit 7, exponent bits 6-3 (bias 7),
+    mantissa bits 2-0; exponent 0 is subnormal (m/8 * 2^-6); S.1111.111 is NaN;
+    there are no infinities (the largest finite magnitude is 448)."""
+    b = np.asarray(bits, dtype=np.int64) & 0xFF
+    sign = np.where(b & 0x80, -1.0, 1.0)
+    e = (b >> 3) & 0xF
+    m = (b & 0x7).astype(np.float64)
+    val = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7.0))
+    val = sign * val
+    return np.where((e == 15) & (m == 7), np.nan, val)
+
+
+def dequant_fp8(bits, scale) -> np.ndarray:
+    """Cached values of an FP8 cache: bits [B, S, Hkv, D] uint8, scale [B, S, Hkv] fp32;
+    value = e4m3(bits) * scale of its (token, KV head) row."""
+    return e4m3_to_float(bits) * _f64(scale)[..., None]
+
+
+def decode_fp8(q, k_bits, v_bits, k_scale, v_scale, kind: str, lengths, sink, scale=None):
+    """One-token decode over an FP8 cache: decode() on the dequantized values."""
+    return decode(q, dequant_fp8(k_bits, k_scale), dequant_fp8(v_bits, v_scale), kind, lengths,
+                  sink, scale)
+
+
+def sparse_decode_fp8(q, k_bits, v_bits, k_scale, v_scale, lengths, recent: int, sel_idx, sink,
+                      scale=None):
+    """Token-level sparse decode over an FP8 cache: sparse_decode() on the dequantized values."""
+    return sparse_decode(q, dequant_fp8(k_bits, k_scale), dequant_fp8(v_bits, v_scale), lengths,
+                         recent, sel_idx, sink, scale)

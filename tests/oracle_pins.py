@@ -344,6 +344,63 @@ def check_multi_decode_matches_prefill(ref):
         raise AssertionError("a ring without room for every draft token's window must be refused")
 
 
+def check_e4m3_decoding(ref):
+    """OCP FP8 E4M3: every one of the 256 byte patterns decodes as torch.float8_e4m3fn
+    does, and the landmarks of the format hold (1.0, the largest 448, the smallest
+    normal 2^-6 and subnormal 2^-9, signed zero, the two NaNs)."""
+    import torch
+    bits = np.arange(256)
+    got = ref.e4m3_to_float(bits)
+    want = torch.from_numpy(bits.astype(np.uint8)).view(torch.float8_e4m3fn).float().numpy().astype(np.float64)
+    assert np.array_equal(np.isnan(got), np.isnan(want))
+    assert np.array_equal(got[~np.isnan(got)], want[~np.isnan(want)])
+    assert got[0x38] == 1.0 and got[0x7E] == 448.0 and got[0xFE] == -448.0
+    assert got[0x08] == 2.0 ** -6 and got[0x01] == 2.0 ** -9 and got[0x07] == 7 * 2.0 ** -9
+    assert got[0x00] == 0.0 and got[0x80] == 0.0 and np.signbit(got[0x80])
+    assert np.isnan(got[0x7F]) and np.isnan(got[0xFF]) and int(np.isnan(got).sum()) == 2
+    assert got[0x40] == 2.0 and got[0x39] == 1.125 and got[0xB8] == -1.0
+
+
+def check_fp8_decode_reduces_to_bf16(ref):
+    """With power-of-two scales, e4m3(b) * s is exact in bf16: FP8 decode and sparse
+    decode over the bytes equal decode / sparse_decode over those bf16 values."""
+    r = _rng(29)
+    B, cap, hq, hkv, d, dv = 2, 40, 4, 2, 16, 8
+    kb = r.integers(0, 256, size=(B, cap, hkv, d))
+    vb = r.integers(0, 256, size=(B, cap, hkv, dv))
+    kb[(kb & 0x7F) == 0x7F] = 0x3C                     # no NaN patterns in a cache
+    vb[(vb & 0x7F) == 0x7F] = 0x3C
+    ks = np.exp2(r.integers(-4, 3, size=(B, cap, hkv))).astype(np.float64)
+    vs = np.exp2(r.integers(-4, 3, size=(B, cap, hkv))).astype(np.float64)
+    kf = ref.e4m3_to_float(kb) * ks[..., None]
+    vf = ref.e4m3_to_float(vb) * vs[..., None]
+    q = r.standard_normal((B, hq, d))
+    sink = r.standard_normal(hq)
+    for kind, L in (("ring", [30, 40]), ("linear", [17, 40])):
+        o1, l1 = ref.decode_fp8(q, kb, vb, ks, vs, kind, L, sink)
+        o2, l2 = ref.decode(q, kf, vf, kind, L, sink)
+        np.testing.assert_array_equal(o1, o2)
+        np.testing.assert_array_equal(l1, l2)
+    sel = np.stack([np.stack([np.sort(r.choice(20, 6, replace=False)) for _ in range(hkv)])
+                    for _ in range(B)])
+    o1, l1 = ref.sparse_decode_fp8(q, kb, vb, ks, vs, [40, 36], 8, sel, sink)
+    o2, l2 = ref.sparse_decode(q, kf, vf, [40, 36], 8, sel, sink)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(l1, l2)
+    # the scale applies per (token, KV head) row: with all scores equal (K bytes 0), doubling
+    # one row's V scale moves exactly the query heads of that KV head in that sequence, by
+    # that row's share of the output
+    k0 = np.zeros_like(kb)
+    vs2 = vs.copy()
+    vs2[0, 5, 1] *= 2.0
+    o3, _ = ref.decode_fp8(q, k0, vb, ks, vs2, "linear", [40, 40], sink)
+    o4, _ = ref.decode_fp8(q, k0, vb, ks, vs, "linear", [40, 40], sink)
+    assert np.array_equal(o3[1], o4[1]) and np.array_equal(o3[0, :2], o4[0, :2])
+    for h in (2, 3):
+        share = 1.0 / (40.0 + np.exp(sink[h]))        # weight of each key, all scores 0
+        np.testing.assert_allclose(o3[0, h] - o4[0, h], share * vf[0, 5, 1], rtol=1e-12, atol=1e-14)
+
+
 def check_sparse_membership(ref):
     """aideepthink.cn §四.3: the key set is the most recent ``recent`` tokens
     plus the selected ones, in one softmax. One-hot values expose membership."""
@@ -423,5 +480,7 @@ ALL_CHECKS = [
     check_decode_matches_prefill,
     check_multi_decode_matches_prefill,
     check_sparse_membership,
+    check_e4m3_decoding,
+    check_fp8_decode_reduces_to_bf16,
     check_golden,
 ]

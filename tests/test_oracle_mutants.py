@@ -42,6 +42,11 @@ MUTANTS = {
                                        "return np.arange(lo, p + 1, dtype=np.int64) - max(0, L - capacity)"),
     "draft causal prefix excludes itself": ("        return np.arange(p + 1, dtype=np.int64)\n",
                                             "        return np.arange(p, dtype=np.int64)\n"),
+    "e4m3 exponent bias 8": ("np.exp2(e.astype(np.float64) - 7.0)", "np.exp2(e.astype(np.float64) - 8.0)"),
+    "e4m3 subnormal scale": ("m / 8.0 * 2.0 ** -6", "m / 8.0 * 2.0 ** -7"),
+    "e4m3 without NaN": ("np.where((e == 15) & (m == 7), np.nan, val)", "val"),
+    "fp8 scale per token only": ("e4m3_to_float(bits) * _f64(scale)[..., None]",
+                                 "e4m3_to_float(bits) * _f64(scale)[..., :1, None]"),
 }
 
 
