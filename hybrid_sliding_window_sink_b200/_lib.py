@@ -27,6 +27,7 @@ STATUS = {0: "MIMO_OK", 1: "MIMO_ERR_NULL", 2: "MIMO_ERR_SHAPE", 3: "MIMO_ERR_UN
 #: Every symbol include/mimo_attn.h declares.
 EXPORTS = ("mimo_attn_prefill", "mimo_attn_decode", "mimo_attn_sparse", "mimo_attn_sparse_noalloc",
            "mimo_attn_decode_mq", "mimo_attn_decode_mq_workspace_size", "mimo_attn_workspace_size",
+           "mimo_attn_decode_fp8", "mimo_attn_sparse_fp8",
            "mimo_attn_check_indices", "mimo_attn_last_device_error", "mimo_status_string",
            "mimo_attn_version")
 
@@ -67,6 +68,8 @@ def lib():
     L.mimo_attn_decode_mq.argtypes = [SP, P, P, P, I, I, LL, P, I, I, P, P, P, P, SZ, P]
     L.mimo_attn_decode_mq_workspace_size.argtypes = [SP, I, I, I, I]
     L.mimo_attn_decode_mq_workspace_size.restype = SZ
+    L.mimo_attn_decode_fp8.argtypes = [SP, P, P, P, P, P, I, I, LL, P, P, P, P, P, SZ, P]
+    L.mimo_attn_sparse_fp8.argtypes = [SP, P, P, P, P, P, I, LL, P, I, P, I, P, P, P, P, SZ, P]
     L.mimo_attn_workspace_size.argtypes = [SP, I, I, I, I, I]
     L.mimo_attn_workspace_size.restype = SZ
     L.mimo_attn_check_indices.argtypes = [SP, P, P, I, I, I, P, P]
@@ -221,6 +224,72 @@ def decode_mq(q, k_cache, v_cache, lengths, sink=None, *, kind="ring", window=12
                                    cap, stride, _ptr(lengths), T, int(window), _ptr(sink), _ptr(out),
                                    _ptr(lse), _ptr(ws), nbytes, _stream(stream))
     _check("mimo_attn_decode_mq", st)
+    return out, lse
+
+
+def _need_fp8(k8, v8, ks, vs):
+    _need(k8, "k_cache", torch.uint8, 4)
+    _need(v8, "v_cache", torch.uint8, 4)
+    _need(ks, "k_scale", torch.float32, 3)
+    _need(vs, "v_scale", torch.float32, 3)
+    if ks.shape != k8.shape[:3] or vs.shape != v8.shape[:3] or k8.shape[:3] != v8.shape[:3]:
+        raise ValueError("FP8 caches and scales disagree in shape")
+
+
+def decode_fp8(q, k8, v8, k_scale, v_scale, lengths, sink=None, *, kind="ring", capacity=None,
+               softmax_scale=0.0, out=None, lse=None, want_lse=True, workspace=None, stream=None):
+    """mimo_attn_decode_fp8. q [B,Hq,192] bf16; k8/v8 [B,stride,Hkv,192/128] uint8 E4M3;
+    k_scale/v_scale [B,stride,Hkv] fp32; value = e4m3(byte) * scale."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need_fp8(k8, v8, k_scale, v_scale)
+    _need(lengths, "lengths", torch.int32, 1)
+    B, hq, dqk = q.shape
+    _, stride, hkv, _ = k8.shape
+    cap = stride if capacity is None else int(capacity)
+    kind_id = {"ring": MIMO_CACHE_RING, "linear": MIMO_CACHE_LINEAR}[kind]
+    if sink is not None:
+        _need(sink, "sink", torch.float32, 1)
+    if out is None:
+        out = torch.empty(B, hq, v8.shape[3], dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty(B, hq, dtype=torch.float32, device=q.device)
+    shape = make_shape(B, 1, hq, hkv, dqk, v8.shape[3], softmax_scale)
+    nbytes = int(lib().mimo_attn_workspace_size(ctypes.byref(shape), MIMO_OP_DECODE, kind_id, cap, 0, 0))
+    ws = _workspace(workspace, nbytes, q.device)
+    st = lib().mimo_attn_decode_fp8(ctypes.byref(shape), _ptr(q), _ptr(k8), _ptr(v8), _ptr(k_scale),
+                                    _ptr(v_scale), kind_id, cap, stride, _ptr(lengths), _ptr(sink),
+                                    _ptr(out), _ptr(lse), _ptr(ws), nbytes, _stream(stream))
+    _check("mimo_attn_decode_fp8", st)
+    return out, lse
+
+
+def sparse_fp8(q, k8, v8, k_scale, v_scale, lengths, sel_idx, sink=None, *, recent=128,
+               capacity=None, softmax_scale=0.0, out=None, lse=None, want_lse=True, workspace=None,
+               stream=None):
+    """mimo_attn_sparse_fp8: sparse() over FP8 linear caches with per-row scales."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need_fp8(k8, v8, k_scale, v_scale)
+    _need(lengths, "lengths", torch.int32, 1)
+    _need(sel_idx, "sel_idx", torch.int32, 3)
+    B, hq, dqk = q.shape
+    _, stride, hkv, _ = k8.shape
+    n_sel = sel_idx.shape[2]
+    cap = stride if capacity is None else int(capacity)
+    if sink is not None:
+        _need(sink, "sink", torch.float32, 1)
+    if out is None:
+        out = torch.empty(B, hq, v8.shape[3], dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty(B, hq, dtype=torch.float32, device=q.device)
+    shape = make_shape(B, 1, hq, hkv, dqk, v8.shape[3], softmax_scale)
+    nbytes = int(lib().mimo_attn_workspace_size(ctypes.byref(shape), MIMO_OP_SPARSE,
+                                                MIMO_CACHE_LINEAR, cap, int(recent), n_sel))
+    ws = _workspace(workspace, nbytes, q.device)
+    st = lib().mimo_attn_sparse_fp8(ctypes.byref(shape), _ptr(q), _ptr(k8), _ptr(v8), _ptr(k_scale),
+                                    _ptr(v_scale), cap, stride, _ptr(lengths), int(recent),
+                                    _ptr(sel_idx), n_sel, _ptr(sink), _ptr(out), _ptr(lse), _ptr(ws),
+                                    nbytes, _stream(stream))
+    _check("mimo_attn_sparse_fp8", st)
     return out, lse
 
 

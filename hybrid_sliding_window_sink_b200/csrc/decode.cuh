@@ -22,6 +22,13 @@
 // owns 16 keys of a subtile: S = Q K^T and O += P V as m16n8k16 bf16 MMAs with the
 // group's (up to 16) query heads as the M dimension; online softmax per warp; the
 // four warp states are merged at the end.
+//
+// FP8 caches (FP8 = true): K and V rows are OCP E4M3 bytes with one fp32 scale per (token,
+// KV head) row for each tensor. Each subtile's bytes and scales are gathered by cp.async
+// into a raw stage, then converted exactly into the MMA layout: K to f16 (E4M3 -> f16 is
+// exact) for an f16 S = Q K^T with Q converted to f16 once, V to bf16 (exact). The K scale
+// multiplies the fp32 score; the V scale multiplies P before it is rounded to bf16 for the
+// PV MMA, while the denominator sums the unscaled P. Q must lie inside the f16 range.
 #pragma once
 
 #include "ptx.cuh"
@@ -38,6 +45,10 @@ constexpr int kVRow = kDV * 2;                     // 256 bytes
 constexpr int kDecStageBytes = kDecSub * (kKRow + kVRow);   // 40960
 constexpr int kDecMaxTokList = 512;                // sparse chunk limit (tokens staged in smem)
 constexpr int kDecSmemBytes = kDecStages * kDecStageBytes + kDecMaxTokList * 4;
+// FP8: one converted stage, two raw stages (bytes + scales), per-subtile scales, token list
+constexpr int kKRow8 = kDQK, kVRow8 = kDV;                    // bytes per cached row
+constexpr int kDecRawBytes = kDecSub * (kKRow8 + kVRow8) + 2 * kDecSub * 4;   // 20992
+constexpr int kDecSmemBytesFp8 = kDecStageBytes + 2 * kDecRawBytes + 2 * kDecSub * 4 + kDecMaxTokList * 4;
 
 enum : int { kModeRing = 0, kModeLinear = 1, kModeSparse = 2 };
 
@@ -53,6 +64,10 @@ struct DecodeParams {
   float* part_ml;             // [B*Hq, nchunks, 2]  (m in log2 units, l)
   float* part_o;              // [B*Hq, nchunks, 128]
   long long seq_stride;       // tokens between sequences
+  const uint8_t* k8;          // FP8 caches: [B, seq_stride, Hkv, 192] / [.., 128] E4M3 bytes
+  const uint8_t* v8;
+  const float* k_scale;       // [B, seq_stride, Hkv] fp32 (FP8 only)
+  const float* v_scale;
   int B, Hq, Hkv, group, cap, mode, chunk, nchunks, recent, n_sel, direct;
   float scale_log2;           // softmax scale * log2(e)
   unsigned* err;
@@ -85,7 +100,33 @@ __device__ __forceinline__ int dec_token(const DecodeParams& p, int b, int g, in
   return x < p.cap - 1 ? x : p.cap - 1;
 }
 
-template <int G>
+// 4-byte cp.async (zero-filled when src_bytes = 0).
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mma_16816_f16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0,
+                                              uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+      "{%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// Two E4M3 bytes (lo = first) -> packed f16x2, exactly.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
+  return r;
+}
+// Packed f16x2 holding E4M3 values (at most 4 significant bits) -> packed bf16x2, exactly.
+__device__ __forceinline__ uint32_t f16x2_to_bf16x2(uint32_t v) {
+  const __half2 h = *reinterpret_cast<const __half2*>(&v);
+  const float2 f = __half22float2(h);
+  return pack_bf16(f.x, f.y);
+}
+
+template <int G, bool FP8 = false>
 __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const DecodeParams p) {
   static_assert(G >= 1 && G <= 16, "group size");
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -100,7 +141,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
   int n_here = nkeys - k_begin;
   n_here = n_here < 0 ? 0 : (n_here < p.chunk ? n_here : p.chunk);
 
-  int* s_tok = reinterpret_cast<int*>(smem + kDecStages * kDecStageBytes);
+  int* s_tok = reinterpret_cast<int*>(smem + (FP8 ? kDecSmemBytesFp8 - kDecMaxTokList * 4
+                                                    : kDecStages * kDecStageBytes));
   if (p.mode == kModeSparse) {
     for (int i = tid; i < n_here; i += kDecThreads) s_tok[i] = dec_token(p, b, g, k_begin + i, nw, L);
     __syncthreads();
@@ -116,7 +158,46 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
     return p.mode == kModeSparse ? s_tok[key] : k_begin + key;
   };
 
+  const uint8_t* kbase8 = p.k8 + g * kKRow8;
+  const uint8_t* vbase8 = p.v8 + g * kVRow8;
+  // FP8: bytes and scales of subtile st into raw stage `stage` (unswizzled rows)
+  auto load_raw = [&](int st, int stage) {
+    const uint32_t r0 = s_base + kDecStageBytes + stage * kDecRawBytes;
+    const uint32_t rK = r0, rV = r0 + kDecSub * kKRow8, rS = rV + kDecSub * kVRow8;
+    const int base = st * kDecSub;
+#pragma unroll
+    for (int i = 0; i < (kDecSub * 12) / kDecThreads; ++i) {      // 6 x 16 B of K per thread
+      const int idx = tid + i * kDecThreads;
+      const int row = idx / 12, u = idx - row * 12;
+      const int key = base + row;
+      const bool ok = key < n_here;
+      const int tok = ok ? token_of(key) : 0;
+      cp_async16(rK + row * kKRow8 + u * 16, kbase8 + (seq0 + tok) * (krow_stride) + u * 16, ok ? 16u : 0u);
+    }
+#pragma unroll
+    for (int i = 0; i < (kDecSub * 8) / kDecThreads; ++i) {       // 4 x 16 B of V per thread
+      const int idx = tid + i * kDecThreads;
+      const int row = idx >> 3, u = idx & 7;
+      const int key = base + row;
+      const bool ok = key < n_here;
+      const int tok = ok ? token_of(key) : 0;
+      cp_async16(rV + row * kVRow8 + u * 16, vbase8 + (seq0 + tok) * (vrow_stride) + u * 16, ok ? 16u : 0u);
+    }
+    {                                                             // one scale per thread
+      const int row = tid & (kDecSub - 1);
+      const bool isv = tid >= kDecSub;
+      const int key = base + row;
+      const bool ok = key < n_here;
+      const int tok = ok ? token_of(key) : 0;
+      const float* src = (isv ? p.v_scale : p.k_scale) + (seq0 + tok) * p.Hkv + g;
+      cp_async4(rS + (isv ? kDecSub * 4 : 0) + row * 4, src, ok ? 4u : 0u);
+    }
+  };
   auto load_sub = [&](int st, int stage) {
+    if (FP8) {
+      load_raw(st, stage);
+      return;
+    }
     const uint32_t sK = s_base + stage * kDecStageBytes;
     const uint32_t sV = sK + kDecSub * kKRow;
     const int base = st * kDecSub;
@@ -161,6 +242,12 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
       qa[kk][2] = r0ok ? *reinterpret_cast<const uint32_t*>(qg + gq * kDQK + d0 + 8) : 0u;
       qa[kk][3] = r1ok ? *reinterpret_cast<const uint32_t*>(qg + (gq + 8) * kDQK + d0 + 8) : 0u;
     }
+    if (FP8) {   // S runs as an f16 MMA against the exactly converted K
+#pragma unroll
+      for (int kk = 0; kk < 12; ++kk)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) qa[kk][j] = pack_f16(bf16_lo(qa[kk][j]), bf16_hi(qa[kk][j]));
+    }
   }
 
   float o[16][4];
@@ -168,10 +255,50 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
   for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
 
+  float* s_ks = reinterpret_cast<float*>(smem + kDecStageBytes + 2 * kDecRawBytes);   // FP8
+  float* s_vs = s_ks + kDecSub;
   for (int st = 0; st < nsub; ++st) {
     cp_async_wait<1>();
     __syncthreads();
-    const uint32_t sK = s_base + (st & 1) * kDecStageBytes;
+    if (FP8) {
+      // raw stage (st & 1) -> converted stage 0: K to f16, V to bf16, scales aside
+      const uint8_t* raw = smem + kDecStageBytes + (st & 1) * kDecRawBytes;
+#pragma unroll
+      for (int i = 0; i < (kDecSub * 12) / kDecThreads; ++i) {
+        const int idx = tid + i * kDecThreads;
+        const int row = idx / 12, u = idx - row * 12;              // 16 bytes -> 2 units
+        const uint4 x = *reinterpret_cast<const uint4*>(raw + row * kKRow8 + u * 16);
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+        uint32_t h[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          h[2 * j] = e4m3x2_to_f16x2(static_cast<uint16_t>(w[j] & 0xFFFFu));
+          h[2 * j + 1] = e4m3x2_to_f16x2(static_cast<uint16_t>(w[j] >> 16));
+        }
+        const uint32_t dst = s_base + row * kKRow;
+        st_shared_v4(dst + (((2 * u) ^ (row & 7)) << 4), h[0], h[1], h[2], h[3]);
+        st_shared_v4(dst + (((2 * u + 1) ^ (row & 7)) << 4), h[4], h[5], h[6], h[7]);
+      }
+#pragma unroll
+      for (int i = 0; i < (kDecSub * 8) / kDecThreads; ++i) {
+        const int idx = tid + i * kDecThreads;
+        const int row = idx >> 3, u = idx & 7;
+        const uint4 x = *reinterpret_cast<const uint4*>(raw + kDecSub * kKRow8 + row * kVRow8 + u * 16);
+        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+        uint32_t h[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          h[2 * j] = f16x2_to_bf16x2(e4m3x2_to_f16x2(static_cast<uint16_t>(w[j] & 0xFFFFu)));
+          h[2 * j + 1] = f16x2_to_bf16x2(e4m3x2_to_f16x2(static_cast<uint16_t>(w[j] >> 16)));
+        }
+        const uint32_t dst = s_base + kDecSub * kKRow + row * kVRow;
+        st_shared_v4(dst + (((2 * u) ^ (row & 7)) << 4), h[0], h[1], h[2], h[3]);
+        st_shared_v4(dst + (((2 * u + 1) ^ (row & 7)) << 4), h[4], h[5], h[6], h[7]);
+      }
+      s_ks[tid] = reinterpret_cast<const float*>(raw + kDecSub * (kKRow8 + kVRow8))[tid];   // K | V
+      __syncthreads();
+    }
+    const uint32_t sK = s_base + (FP8 ? 0 : (st & 1) * kDecStageBytes);
     const uint32_t sV = sK + kDecSub * kKRow;
     const int mi = lane >> 3, r8 = lane & 7;
 
@@ -185,8 +312,13 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
         const int unit = 2 * kk + (mi & 1);
         uint32_t b00, b01, b10, b11;
         ldmatrix_x4(rowaddr + ((unit ^ (krow & 7)) << 4), b00, b01, b10, b11);
-        mma_16816(sacc[0], qa[kk], b00, b01);
-        mma_16816(sacc[1], qa[kk], b10, b11);
+        if (FP8) {
+          mma_16816_f16(sacc[0], qa[kk], b00, b01);
+          mma_16816_f16(sacc[1], qa[kk], b10, b11);
+        } else {
+          mma_16816(sacc[0], qa[kk], b00, b01);
+          mma_16816(sacc[1], qa[kk], b10, b11);
+        }
       }
     }
 
@@ -198,7 +330,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const bool ok = keybase + nt * 8 + (e & 1) < n_here;
-        s[nt][e] = ok ? sacc[nt][e] * p.scale_log2 : -INFINITY;
+        const float ksc = FP8 ? s_ks[keybase - st * kDecSub + nt * 8 + (e & 1)] : 1.f;
+        s[nt][e] = ok ? sacc[nt][e] * ksc * p.scale_log2 : -INFINITY;
       }
     }
     float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
@@ -227,6 +360,15 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
     for (int j = 0; j < 16; ++j) {
       o[j][0] *= al0; o[j][1] *= al0;
       o[j][2] *= al1; o[j][3] *= al1;
+    }
+    if (FP8) {   // fold each key's V scale into P (the denominator used the unscaled P)
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        const int kl = keybase - st * kDecSub + nt * 8;
+        const float v0 = s_vs[kl], v1 = s_vs[kl + 1];
+        pv[nt][0] *= v0; pv[nt][1] *= v1;
+        pv[nt][2] *= v0; pv[nt][3] *= v1;
+      }
     }
     uint32_t pa[4];
     pa[0] = pack_bf16(pv[0][0], pv[0][1]);

@@ -257,16 +257,16 @@ DecodePlan plan_decode(const mimo_shape* s, int mode, int cap, int recent, int n
   return pl;
 }
 
-template <int G>
+template <int G, bool FP8 = false>
 mimo_status launch_decode_g(DecodeParams prm, cudaStream_t st) {
-  auto kern = mimo::decode_split_kernel<G>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, mimo::kDecSmemBytes) !=
-      cudaSuccess) {
+  auto kern = mimo::decode_split_kernel<G, FP8>;
+  const int smem = FP8 ? mimo::kDecSmemBytesFp8 : mimo::kDecSmemBytes;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
     cudaGetLastError();
     return MIMO_ERR_CUDA;
   }
   dim3 grid(prm.nchunks, prm.Hkv, prm.B);
-  kern<<<grid, mimo::kDecThreads, mimo::kDecSmemBytes, st>>>(prm);
+  kern<<<grid, mimo::kDecThreads, smem, st>>>(prm);
   if (cudaGetLastError() != cudaSuccess) return MIMO_ERR_CUDA;
   if (!prm.direct) {
     mimo::decode_combine_kernel<<<prm.B * prm.Hq, mimo::kDV, 0, st>>>(prm);
@@ -275,13 +275,17 @@ mimo_status launch_decode_g(DecodeParams prm, cudaStream_t st) {
   return MIMO_OK;
 }
 
+// FP8 caches: kc / vc are E4M3 bytes and ks / vs their per-(token, KV head) fp32 scales.
 mimo_status run_decode(const mimo_shape* s, int mode, const void* q, const void* kc, const void* vc,
                        int cap, long long stride, const int* lengths, int recent, const int* sel,
                        int n_sel, const float* sink, void* out, float* lse, void* ws, size_t ws_bytes,
-                       void* stream) {
+                       void* stream, bool fp8 = false, const float* ks = nullptr,
+                       const float* vs = nullptr) {
   mimo_status e = check_heads(s);
   if (e != MIMO_OK) return e;
   if (!q || !kc || !vc || !lengths || !out) return MIMO_ERR_NULL;
+  if (fp8 && (!ks || !vs)) return MIMO_ERR_NULL;
+  if (fp8 && (!aligned(ks, 4) || !aligned(vs, 4))) return MIMO_ERR_ALIGN;
   if (mode == mimo::kModeSparse && n_sel > 0 && !sel) return MIMO_ERR_NULL;
   if (cap < 1 || stride < cap) return MIMO_ERR_SHAPE;
   if (mode == mimo::kModeSparse && (recent < 0 || n_sel < 0)) return MIMO_ERR_SHAPE;
@@ -297,8 +301,15 @@ mimo_status run_decode(const mimo_shape* s, int mode, const void* q, const void*
   if (ws && !aligned(ws, 16)) return MIMO_ERR_ALIGN;
   DecodeParams prm{};
   prm.q = static_cast<const __nv_bfloat16*>(q);
-  prm.k = static_cast<const __nv_bfloat16*>(kc);
-  prm.v = static_cast<const __nv_bfloat16*>(vc);
+  if (fp8) {
+    prm.k8 = static_cast<const uint8_t*>(kc);
+    prm.v8 = static_cast<const uint8_t*>(vc);
+    prm.k_scale = ks;
+    prm.v_scale = vs;
+  } else {
+    prm.k = static_cast<const __nv_bfloat16*>(kc);
+    prm.v = static_cast<const __nv_bfloat16*>(vc);
+  }
   prm.lengths = lengths;
   prm.sel = sel;
   prm.sink = sink;
@@ -327,6 +338,15 @@ mimo_status run_decode(const mimo_shape* s, int mode, const void* q, const void*
   if (!prm.err) return MIMO_ERR_CUDA;
   if (s->n_kv_heads > 65535) return MIMO_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (fp8) {
+    switch (prm.group) {
+      case 1: return launch_decode_g<1, true>(prm, st);
+      case 2: return launch_decode_g<2, true>(prm, st);
+      case 4: return launch_decode_g<4, true>(prm, st);
+      case 8: return launch_decode_g<8, true>(prm, st);
+      default: return launch_decode_g<16, true>(prm, st);
+    }
+  }
   switch (prm.group) {
     case 1: return launch_decode_g<1>(prm, st);
     case 2: return launch_decode_g<2>(prm, st);
@@ -520,6 +540,29 @@ size_t mimo_attn_decode_mq_workspace_size(const mimo_shape* s, int cache_kind, i
   if (check_mq(s, cache_kind, cache_capacity, q_len, window) != MIMO_OK) return 0;
   const int mode = cache_kind == MIMO_CACHE_RING ? mimo::kModeRing : mimo::kModeLinear;
   return plan_decode_mq(s, mode, cache_capacity, q_len, window, sm_count_for(current_device())).bytes;
+}
+
+mimo_status mimo_attn_decode_fp8(const mimo_shape* s, const void* q, const void* k_cache,
+                                 const void* v_cache, const float* k_scale, const float* v_scale,
+                                 int cache_kind, int cache_capacity, long long seq_stride_tokens,
+                                 const int* lengths, const float* sink, void* out, float* lse,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  if (cache_kind != MIMO_CACHE_RING && cache_kind != MIMO_CACHE_LINEAR) return MIMO_ERR_SHAPE;
+  const int mode = cache_kind == MIMO_CACHE_RING ? mimo::kModeRing : mimo::kModeLinear;
+  return run_decode(s, mode, q, k_cache, v_cache, cache_capacity, seq_stride_tokens, lengths, 0,
+                    nullptr, 0, sink, out, lse, workspace, workspace_bytes, stream, true, k_scale,
+                    v_scale);
+}
+
+mimo_status mimo_attn_sparse_fp8(const mimo_shape* s, const void* q, const void* k_cache,
+                                 const void* v_cache, const float* k_scale, const float* v_scale,
+                                 int cache_capacity, long long seq_stride_tokens, const int* lengths,
+                                 int recent, const int* sel_idx, int n_sel, const float* sink,
+                                 void* out, float* lse, void* workspace, size_t workspace_bytes,
+                                 void* stream) {
+  return run_decode(s, mimo::kModeSparse, q, k_cache, v_cache, cache_capacity, seq_stride_tokens,
+                    lengths, recent, sel_idx, n_sel, sink, out, lse, workspace, workspace_bytes,
+                    stream, true, k_scale, v_scale);
 }
 
 size_t mimo_attn_workspace_size(const mimo_shape* s, int op, int cache_kind, int cache_capacity,

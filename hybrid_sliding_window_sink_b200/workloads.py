@@ -151,6 +151,25 @@ def decode_mq_inputs(batch, q_len, hq, hkv, capacity, lengths, *, seed, device="
     return inp
 
 
+def fp8_cache(x):
+    """Quantizes a bf16/fp32 cache [B, S, Hkv, D] to E4M3 bytes with one fp32 scale per
+    (token, KV head) row (amax / 448, 1 for an all-zero row), the way a serving stack would
+    write it. Returns (bytes uint8 [B, S, Hkv, D], scale fp32 [B, S, Hkv])."""
+    xf = x.float()
+    amax = xf.abs().amax(dim=-1)
+    scale = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+    q = (xf / scale[..., None]).to(torch.float8_e4m3fn)
+    return q.view(torch.uint8), scale.contiguous()
+
+
+def decode_fp8_inputs(batch, hq, hkv, capacity, lengths, *, seed, device="cpu"):
+    """decode_inputs (same draws) plus k8/v8 E4M3 caches and k_scale/v_scale from fp8_cache."""
+    inp = decode_inputs(batch, hq, hkv, capacity, lengths, seed=seed, device=device)
+    inp["k8"], inp["k_scale"] = fp8_cache(inp["k_cache"])
+    inp["v8"], inp["v_scale"] = fp8_cache(inp["v_cache"])
+    return inp
+
+
 def sorted_unique_indices(batch, hkv, n_sel, hi_excl, *, seed):
     """[B, Hkv, n_sel] int32, each row sorted unique uniform in [0, hi_excl[b])."""
     g = _gen(seed + 13, "cpu")

@@ -192,6 +192,36 @@ mimo_status mimo_attn_decode_mq(const mimo_shape* shape, const void* q, const vo
 size_t mimo_attn_decode_mq_workspace_size(const mimo_shape* shape, int cache_kind,
                                           int cache_capacity, int q_len, int window);
 
+/*
+ * Decode and token-level sparse decode over FP8 KV caches. The pages size their KV caches
+ * in FP8 but state no scaling scheme; this library's scheme: K and V hold OCP FP8 E4M3
+ * bytes (bias 7, no infinities, S.1111.111 is NaN) and each (token, KV head) row has one
+ * fp32 scale per tensor; the cached value is e4m3(byte) * scale. Attention is that of
+ * mimo_attn_decode / mimo_attn_sparse on those values.
+ *
+ *  k_cache [B, seq_stride_tokens, Hkv, 192] uint8 device (E4M3), rows 16-byte aligned
+ *  v_cache [B, seq_stride_tokens, Hkv, 128] uint8 device (E4M3)
+ *  k_scale, v_scale [B, seq_stride_tokens, Hkv] fp32 device, 4-byte aligned
+ *  every other argument, the workspace size (mimo_attn_workspace_size with the same op,
+ *  kind and sizes) and the errors: as mimo_attn_decode / mimo_attn_sparse; MIMO_ERR_NULL
+ *  also for a missing scale array.
+ *
+ * The E4M3 bytes are converted exactly (K to f16, V to bf16); the K scale multiplies the
+ * fp32 score and the V scale multiplies P before its bf16 rounding. q must lie inside the
+ * f16 range (|q| < 65504) because S = Q K^T runs as an f16 MMA.
+ */
+mimo_status mimo_attn_decode_fp8(const mimo_shape* shape, const void* q, const void* k_cache,
+                                 const void* v_cache, const float* k_scale, const float* v_scale,
+                                 int cache_kind, int cache_capacity, long long seq_stride_tokens,
+                                 const int* lengths, const float* sink, void* out, float* lse,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+mimo_status mimo_attn_sparse_fp8(const mimo_shape* shape, const void* q, const void* k_cache,
+                                 const void* v_cache, const float* k_scale, const float* v_scale,
+                                 int cache_capacity, long long seq_stride_tokens, const int* lengths,
+                                 int recent, const int* sel_idx, int n_sel, const float* sink,
+                                 void* out, float* lse, void* workspace, size_t workspace_bytes,
+                                 void* stream);
+
 /* Bytes of device workspace mimo_attn_decode / mimo_attn_sparse need for these sizes
  * on the current device (0 when none is needed). Returns 0 for invalid arguments. */
 size_t mimo_attn_workspace_size(const mimo_shape* shape, int op, int cache_kind,
