@@ -410,6 +410,80 @@ def bench_mtp_step(steps, warmup, peaks, tag, dev, stream, q_len=4):
     return res
 
 
+def fp8_decode_layer_bytes(lengths, hq, hkv, kind, cap):
+    """Algorithmic bytes of one FP8-cache decode layer: E4M3 K/V rows (320 B) plus the two
+    fp32 row scales per (token, KV head), and q, out, lse."""
+    L = np.asarray(lengths, dtype=np.int64)
+    keys = np.minimum(L, cap) if kind == "ring" else L
+    kv = int(keys.sum()) * hkv * (wl.DQK + wl.DV + 8)
+    B = len(L)
+    return float(kv + B * hq * wl.DQK * 2 + B * hq * wl.DV * 2 + B * hq * 4 + hq * 4 + B * 4)
+
+
+def _random_e4m3(shape, g, dev):
+    """Random E4M3 bytes (NaN patterns replaced by 0) for timing runs."""
+    b = torch.randint(0, 256, shape, generator=g, device=dev, dtype=torch.int32)
+    b = torch.where((b & 0x7F) == 0x7F, torch.zeros_like(b), b)
+    return b.to(torch.uint8)
+
+
+def bench_fp8_decode_step(steps, warmup, peaks, tag, dev, stream):
+    """The hybrid decode step of bench_decode_step over FP8 caches (E4M3 K/V with
+    per-(token, KV head) fp32 scales): 39 SWA rings of 128 slots, 9 GA layers on one padded
+    linear cache of 131072 slots, B=64, same lengths."""
+    from hybrid_sliding_window_sink_b200 import _lib
+    cs, cg = wl.HYBRID_DECODE_SWA, wl.HYBRID_DECODE_GA
+    L = wl.lengths_uniform(cs.batch, cs.min_len, cs.max_len, seed=cs.seed)
+    Ld = L.to(dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(cs.seed + 9)
+    mk_scale = lambda *sh: torch.empty(*sh, device=dev).uniform_(0.002, 0.01, generator=g)  # noqa: E731
+    ga = (_random_e4m3((cg.batch, cg.capacity, cg.hkv, wl.DQK), g, dev),
+          _random_e4m3((cg.batch, cg.capacity, cg.hkv, wl.DV), g, dev),
+          mk_scale(cg.batch, cg.capacity, cg.hkv), mk_scale(cg.batch, cg.capacity, cg.hkv))
+    layers = []
+    for kind in wl.layer_pattern():
+        q = torch.randn(cs.batch, cs.hq, wl.DQK, generator=g, device=dev).to(torch.bfloat16)
+        sink = torch.randn(cs.hq, generator=g, device=dev)
+        if kind == 1:
+            cache = (_random_e4m3((cs.batch, cs.capacity, cs.hkv, wl.DQK), g, dev),
+                     _random_e4m3((cs.batch, cs.capacity, cs.hkv, wl.DV), g, dev),
+                     mk_scale(cs.batch, cs.capacity, cs.hkv), mk_scale(cs.batch, cs.capacity, cs.hkv))
+        else:
+            cache = ga
+        out = torch.empty(cs.batch, cs.hq, wl.DV, dtype=torch.bfloat16, device=dev)
+        lse = torch.empty(cs.batch, cs.hq, dtype=torch.float32, device=dev)
+        layers.append((kind, q, cache, sink, out, lse))
+    nws = _lib.workspace_size(cg.batch, cg.hq, cg.hkv, op=_lib.MIMO_OP_DECODE,
+                              kind=_lib.MIMO_CACHE_LINEAR, capacity=cg.capacity)
+    ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
+
+    def run_layer(lay):
+        kind, q, (k8, v8, ks, vs), sink, out, lse = lay
+        _lib.decode_fp8(q, k8, v8, ks, vs, Ld, sink, kind="ring" if kind == 1 else "linear",
+                        out=out, lse=lse, workspace=ws, stream=stream)
+
+    ms = timed(lambda: [run_layer(l) for l in layers], steps, warmup, stream)
+    Ls = L.tolist()
+    b_swa = fp8_decode_layer_bytes(Ls, cs.hq, cs.hkv, "ring", cs.capacity)
+    b_ga = fp8_decode_layer_bytes(Ls, cg.hq, cg.hkv, "linear", cg.capacity)
+    total = 39 * b_swa + 9 * b_ga
+    ms_ga = timed(lambda: [run_layer(l) for l in layers if l[0] == 0], steps, 1, stream) / (steps * 9)
+    ms_swa = timed(lambda: [run_layer(l) for l in layers if l[0] == 1], steps, 1, stream) / (steps * 39)
+    res = {
+        "value": round(total / (ms / steps * 1e-3) / 1e9, 1), "unit": "GB/s",
+        "ms_per_step": round(ms / steps, 4), "bytes_per_step": total,
+        "launches_per_step": 39 + 9 * 2,
+        "ga_layer": roofline_hbm(b_ga, ms_ga, peaks, tag),
+        "swa_layer": roofline_hbm(b_swa, ms_swa, peaks, tag),
+        "roofline": roofline_hbm(total, ms / steps, peaks, tag),
+        "ms_ga_layer": round(ms_ga, 4), "ms_swa_layer": round(ms_swa, 5),
+        "cache": "E4M3 K/V + fp32 scale per (token, KV head); 39 distinct 128-slot rings; one padded GA cache",
+    }
+    del layers, ga, ws
+    return res
+
+
 def bench_sparse(steps, warmup, peaks, tag, dev, stream, calls=16):
     """Token-level sparse decode: ``calls`` independent calls (distinct q and index sets,
     >= 385 MB of gathered rows in all, more than L2) per step, captured in a CUDA graph."""
@@ -580,6 +654,12 @@ def main():
             torch.cuda.empty_cache()
         except Exception as e:
             wls["hybrid_decode_step"] = {"error": repr(e)}
+        try:
+            wls["fp8_decode_step"] = bench_fp8_decode_step(max(3, ksteps), 3, peaks, tag, dev, stream)
+            wls["fp8_decode_step"]["workload"] = "hybrid decode step over FP8 caches, 48 layers, B=64"
+            torch.cuda.empty_cache()
+        except Exception as e:
+            wls["fp8_decode_step"] = {"error": repr(e)}
         try:
             wls["mtp_decode_step"] = bench_mtp_step(max(3, ksteps), 3, peaks, tag, dev, stream)
             wls["mtp_decode_step"]["workload"] = "MTP verification step (1+3 tokens), 48 layers, B=64"

@@ -297,6 +297,10 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
       }
       s_ks[tid] = reinterpret_cast<const float*>(raw + kDecSub * (kKRow8 + kVRow8))[tid];   // K | V
       __syncthreads();
+      // raw stage (st & 1) is consumed: refill it now; the converted stage is protected by the
+      // barrier at the top of the next iteration
+      if (st + 2 < nsub) load_sub(st + 2, st & 1);
+      cp_async_commit();
     }
     const uint32_t sK = s_base + (FP8 ? 0 : (st & 1) * kDecStageBytes);
     const uint32_t sV = sK + kDecSub * kKRow;
@@ -389,9 +393,11 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
         mma_16816(o[2 * jp + 1], pa, v2, v3);
       }
     }
-    __syncthreads();
-    if (st + 2 < nsub) load_sub(st + 2, st & 1);
-    cp_async_commit();
+    if (!FP8) {
+      __syncthreads();
+      if (st + 2 < nsub) load_sub(st + 2, st & 1);
+      cp_async_commit();
+    }
   }
   cp_async_wait<0>();
 

@@ -13,6 +13,8 @@ Cases:
   sparse_b8_l65536      token-level sparse decode, B=8, L=65536, recent 128 + 1024 selected
   mtp_linear_b64_l16k   multi-query (1 + 3 draft tokens) GA decode, B=64, linear cache of 16384
                         tokens (all full), 64 Q / 4 KV heads
+  fp8_linear_b64_l16k   GA decode over an FP8 (E4M3 + per-row scale) linear cache, B=64, 16384
+                        tokens (all full), 64 Q / 4 KV heads
 Prints the mean time per call over --reps calls (after two warm-up calls).
 """
 
@@ -63,6 +65,14 @@ def _case(name, dev):
         ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
         return lambda: _lib.decode_mq(d["q_mq"], d["k_cache"], d["v_cache"], d["lengths"], d["sink"],
                                       kind="linear", window=0, workspace=ws)
+    if name == "fp8_linear_b64_l16k":
+        d = wl.decode_fp8_inputs(64, 64, 4, 16384, [16384] * 64, seed=11, device=dev)
+        del d["k_cache"], d["v_cache"]
+        ws = torch.empty(_lib.workspace_size(64, 64, 4, op=_lib.MIMO_OP_DECODE,
+                                             kind=_lib.MIMO_CACHE_LINEAR, capacity=16384),
+                         dtype=torch.uint8, device=dev)
+        return lambda: _lib.decode_fp8(d["q"], d["k8"], d["v8"], d["k_scale"], d["v_scale"],
+                                       d["lengths"], d["sink"], kind="linear", workspace=ws)
     raise SystemExit(f"unknown case {name}")
 
 
