@@ -399,7 +399,8 @@ def bench_mtp_step(steps, warmup, peaks, tag, dev, stream, q_len=4):
         "value": round(total / (ms / steps * 1e-3) / 1e9, 1), "unit": "GB/s",
         "ms_per_step": round(ms / steps, 4), "bytes_per_step": total, "q_len": q_len,
         "launches_per_step": 39 + 9 * 2,
-        "ga_layer": roofline_hbm(b_ga, ms_ga, peaks, tag),
+        "ga_layer": roofline_hbm(b_ga, ms_ga, peaks, tag,
+                                 traffic_for("decode_mq_linear", int(sum(Ls)) * cg.hkv)),
         "swa_layer": roofline_hbm(b_swa, ms_swa, peaks, tag),
         "roofline": roofline_hbm(total, ms / steps, peaks, tag),
         "ms_ga_layer": round(ms_ga, 4), "ms_swa_layer": round(ms_swa, 5),
@@ -474,7 +475,8 @@ def bench_fp8_decode_step(steps, warmup, peaks, tag, dev, stream):
         "value": round(total / (ms / steps * 1e-3) / 1e9, 1), "unit": "GB/s",
         "ms_per_step": round(ms / steps, 4), "bytes_per_step": total,
         "launches_per_step": 39 + 9 * 2,
-        "ga_layer": roofline_hbm(b_ga, ms_ga, peaks, tag),
+        "ga_layer": roofline_hbm(b_ga, ms_ga, peaks, tag,
+                                 traffic_for("decode_split_fp8_linear", int(sum(Ls)) * cg.hkv)),
         "swa_layer": roofline_hbm(b_swa, ms_swa, peaks, tag),
         "roofline": roofline_hbm(total, ms / steps, peaks, tag),
         "ms_ga_layer": round(ms_ga, 4), "ms_swa_layer": round(ms_swa, 5),
