@@ -41,6 +41,12 @@ Readings where the pages are silent (each also listed in the design notes):
 * Multi-query decode: the T newest tokens of a sequence (positions L-T .. L-1, all
   already written to the cache) are verified together; each has its own window
   (SWA) or causal prefix (GA), exactly as the same rows of a prefill would.
+* Chunked prefill (youngju.dev "mimo-v25-inference-optimization", serving section: long
+  prompts are prefilled in chunks): a chunk of n tokens at positions off .. off+n-1 attends
+  the keys 0 .. off+n-1 exactly as those rows of a whole-sequence prefill would; the prefix
+  keys may come from a KV cache (already rotated) or un-rotated; the chunk's own keys are
+  un-rotated. Appending a chunk to a cache stores its rotated K and its V at slot
+  p mod capacity (ring) or p (linear) for each of its positions p.
 * FP8 KV cache (the pages size their KV caches in FP8 but give no scaling scheme):
   K and V bytes are OCP FP8 E4M3 (bias 7, no infinities, S.1111.111 is NaN), each
   (token, KV head) row carries one fp32 scale per tensor, and the cached value is
@@ -65,6 +71,8 @@ __all__ = [
     "decode_multi",
     "sparse_decode",
     "sparse_key_set",
+    "prefill_chunk",
+    "cache_append",
     "e4m3_to_float",
     "dequant_fp8",
     "decode_fp8",
@@ -406,6 +414,72 @@ def combine_partials(parts, sink):
         L += math.exp(float(sink) - M)
     o = sum(oc * math.exp(m - M) for m, _, oc in parts) / L
     return o, M + math.log(L)
+
+
+# --------------------------------------------------------------------------
+# Chunked prefill over a KV prefix, and appending a chunk to a cache
+# --------------------------------------------------------------------------
+
+def prefill_chunk(q, k, v, pos_offset: int, k_prefix_rotated: bool, sink, window: int,
+                  rope_theta: float, rot_dims: int, scale: float | None = None):
+    """Sink attention of a chunk of n query tokens at positions off .. off+n-1.
+
+    q: [B, n, Hq, Dqk] (un-rotated); k: [B, off+n, Hkv, Dqk], v: [B, off+n, Hkv, Dv] hold
+    every key position 0 .. off+n-1. Key rows at positions < off are used as stored when
+    ``k_prefix_rotated`` (a cache holds rotated K) and rotated otherwise; the chunk's key
+    rows (positions >= off) are rotated. Query i of the chunk is rotated at position
+    off + i and attends window_keys(off + i, window, off + n).
+    Returns (o [B, n, Hq, Dv], lse [B, Hq, n]).
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, n, Hq, D = q.shape
+    nk, Hkv = k.shape[1], k.shape[2]
+    off = int(pos_offset)
+    if nk != off + n or v.shape[1] != nk:
+        raise ValueError("keys must cover positions 0 .. pos_offset + n - 1")
+    group = Hq // Hkv
+    sc = _scale(scale, D)
+    kpos = np.arange(nk, dtype=np.float64)
+    kr = np.stack([rope(k[b], kpos, rope_theta, rot_dims) for b in range(B)])
+    if k_prefix_rotated:
+        kr[:, :off] = k[:, :off]
+    qpos = off + np.arange(n, dtype=np.float64)
+    qr = np.stack([rope(q[b], qpos, rope_theta, rot_dims) for b in range(B)])
+    o = np.zeros((B, n, Hq, v.shape[-1]))
+    lse = np.zeros((B, Hq, n))
+    for b in range(B):
+        for h in range(Hq):
+            g = h // group
+            for i in range(n):
+                keys = window_keys(off + i, window, nk)
+                o[b, i, h], lse[b, h, i] = attend_row(qr[b, i, h], kr[b, :, g, :], v[b, :, g, :],
+                                                      keys, None if sink is None else float(_f64(sink)[h]), sc)
+    return o, lse
+
+
+def cache_append(k_chunk, v_chunk, pos_offset: int, rope_theta: float, rot_dims: int, kind: str,
+                 k_cache, v_cache):
+    """Copies of the caches [B, cap, Hkv, D] after appending a chunk of n tokens at
+    positions off .. off+n-1: K rotated at its position, V as is, at slot p mod cap
+    (ring) or p (linear; needs off + n <= cap). Returns (k_cache', v_cache')."""
+    kc, vc = _f64(k_cache).copy(), _f64(v_cache).copy()
+    kn, vn = _f64(k_chunk), _f64(v_chunk)
+    B, n = kn.shape[0], kn.shape[1]
+    cap = kc.shape[1]
+    off = int(pos_offset)
+    if kind == "linear" and off + n > cap:
+        raise ValueError("linear cache too small")
+    if kind not in ("ring", "linear"):
+        raise ValueError(kind)
+    pos = off + np.arange(n, dtype=np.float64)
+    for b in range(B):
+        kr = rope(kn[b], pos, rope_theta, rot_dims)
+        for i in range(n):
+            p = off + i
+            slot = p % cap if kind == "ring" else p
+            kc[b, slot] = kr[i]
+            vc[b, slot] = vn[b, i]
+    return kc, vc
 
 
 # --------------------------------------------------------------------------

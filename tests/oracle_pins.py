@@ -344,6 +344,46 @@ def check_multi_decode_matches_prefill(ref):
         raise AssertionError("a ring without room for every draft token's window must be refused")
 
 
+def check_chunked_prefill_matches_whole(ref):
+    """Chunked prefill (youngju.dev "mimo-v25-inference-optimization", serving section):
+    cutting a sequence into chunks, each chunk attending the prefix (from a cache holding
+    rotated K, or un-rotated) plus itself, reproduces the whole-sequence prefill row for row
+    (SWA and GA), and appending each chunk to a ring or linear cache leaves exactly the
+    rotated K / V that make a following decode equal the next prefill row."""
+    n, hq, hkv, d, dv = 61, 4, 2, 16, 8
+    q, k, v, sink = _rand_prefill(31, n=n, hq=hq, hkv=hkv, d=d, dv=dv)
+    pos = np.arange(n, dtype=np.float64)
+    kr = ref.rope(k[0], pos, 1e4, 8)[None]
+    for window in (9, 0):
+        o_full, l_full = ref.prefill(q, k, v, sink, window, 1e4, 8)
+        for cuts in ((0, 61), (0, 20, 41, 61), (0, 1, 2, 60, 61), (0, 33, 61)):
+            for a, b in zip(cuts[:-1], cuts[1:]):
+                for rotated in (True, False):
+                    kk = k[:, :b].copy()
+                    if rotated:
+                        kk[:, :a] = kr[:, :a]
+                    o, l = ref.prefill_chunk(q[:, a:b], kk, v[:, :b], a, rotated, sink, window, 1e4, 8)
+                    np.testing.assert_allclose(o, o_full[:, a:b], rtol=1e-11, atol=1e-12)
+                    np.testing.assert_allclose(l, l_full[:, :, a:b], rtol=0, atol=1e-11)
+    # cache write-back: chunks appended to a ring of 12 slots and to a linear cache
+    for kind, cap in (("ring", 12), ("linear", 64)):
+        kc = np.zeros((1, cap, hkv, d))
+        vc = np.zeros((1, cap, hkv, dv))
+        for a, b in ((0, 20), (20, 41), (41, 50)):
+            kc, vc = ref.cache_append(k[:, a:b], v[:, a:b], a, 1e4, 8, kind, kc, vc)
+        L = 50
+        for p in range(max(0, L - cap), L):
+            slot = p % cap if kind == "ring" else p
+            np.testing.assert_allclose(kc[0, slot], kr[0, p], rtol=0, atol=1e-15)
+            np.testing.assert_array_equal(vc[0, slot], v[0, p])
+        qr = ref.rope(q[0, L - 1:L], pos[L - 1:L], 1e4, 8)
+        W = cap if kind == "ring" else 0
+        o_pf, l_pf = ref.prefill(q[:, :L], k[:, :L], v[:, :L], sink, W, 1e4, 8)
+        o, l = ref.decode(qr, kc, vc, kind, [L], sink)
+        np.testing.assert_allclose(o[0], o_pf[0, L - 1], rtol=1e-11, atol=1e-12)
+        np.testing.assert_allclose(l[0], l_pf[0, :, L - 1], rtol=0, atol=1e-11)
+
+
 def check_e4m3_decoding(ref):
     """OCP FP8 E4M3: every one of the 256 byte patterns decodes as torch.float8_e4m3fn
     does, and the landmarks of the format hold (1.0, the largest 448, the smallest
@@ -479,6 +519,7 @@ ALL_CHECKS = [
     check_split_combine,
     check_decode_matches_prefill,
     check_multi_decode_matches_prefill,
+    check_chunked_prefill_matches_whole,
     check_sparse_membership,
     check_e4m3_decoding,
     check_fp8_decode_reduces_to_bf16,

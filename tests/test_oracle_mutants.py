@@ -42,6 +42,15 @@ MUTANTS = {
                                        "return np.arange(lo, p + 1, dtype=np.int64) - max(0, L - capacity)"),
     "draft causal prefix excludes itself": ("        return np.arange(p + 1, dtype=np.int64)\n",
                                             "        return np.arange(p, dtype=np.int64)\n"),
+    "chunk queries at chunk-relative positions": ("    qpos = off + np.arange(n, dtype=np.float64)\n",
+                                                  "    qpos = np.arange(n, dtype=np.float64)\n"),
+    "chunk window measured on the chunk only": ("                keys = window_keys(off + i, window, nk)\n",
+                                                "                keys = window_keys(off + i, window, nk)[-(i + 1):]\n"),
+    "cached prefix rotated twice": ("    if k_prefix_rotated:\n        kr[:, :off] = k[:, :off]\n",
+                                    "    if False:\n        kr[:, :off] = k[:, :off]\n"),
+    "appended K left un-rotated": ("            kc[b, slot] = kr[i]\n", "            kc[b, slot] = kn[b, i]\n"),
+    "ring append without modulo": ("            slot = p % cap if kind == \"ring\" else p\n",
+                                   "            slot = min(p, cap - 1)\n"),
     "e4m3 exponent bias 8": ("np.exp2(e.astype(np.float64) - 7.0)", "np.exp2(e.astype(np.float64) - 8.0)"),
     "e4m3 subnormal scale": ("m / 8.0 * 2.0 ** -6", "m / 8.0 * 2.0 ** -7"),
     "e4m3 without NaN": ("np.where((e == 15) & (m == 7), np.nan, val)", "val"),
