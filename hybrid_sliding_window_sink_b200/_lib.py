@@ -27,7 +27,8 @@ STATUS = {0: "MIMO_OK", 1: "MIMO_ERR_NULL", 2: "MIMO_ERR_SHAPE", 3: "MIMO_ERR_UN
 #: Every symbol include/mimo_attn.h declares.
 EXPORTS = ("mimo_attn_prefill", "mimo_attn_decode", "mimo_attn_sparse", "mimo_attn_sparse_noalloc",
            "mimo_attn_decode_mq", "mimo_attn_decode_mq_workspace_size", "mimo_attn_workspace_size",
-           "mimo_attn_decode_fp8", "mimo_attn_sparse_fp8",
+           "mimo_attn_decode_fp8", "mimo_attn_sparse_fp8", "mimo_attn_prefill_chunk",
+           "mimo_attn_cache_append",
            "mimo_attn_check_indices", "mimo_attn_last_device_error", "mimo_status_string",
            "mimo_attn_version")
 
@@ -68,6 +69,8 @@ def lib():
     L.mimo_attn_decode_mq.argtypes = [SP, P, P, P, I, I, LL, P, I, I, P, P, P, P, SZ, P]
     L.mimo_attn_decode_mq_workspace_size.argtypes = [SP, I, I, I, I]
     L.mimo_attn_decode_mq_workspace_size.restype = SZ
+    L.mimo_attn_prefill_chunk.argtypes = [SP, P, P, P, I, I, P, I, F, I, P, P, P]
+    L.mimo_attn_cache_append.argtypes = [SP, P, P, I, F, I, I, P, P, I, LL, P]
     L.mimo_attn_decode_fp8.argtypes = [SP, P, P, P, P, P, I, I, LL, P, P, P, P, P, SZ, P]
     L.mimo_attn_sparse_fp8.argtypes = [SP, P, P, P, P, P, I, LL, P, I, P, I, P, P, P, P, SZ, P]
     L.mimo_attn_workspace_size.argtypes = [SP, I, I, I, I, I]
@@ -193,6 +196,53 @@ def decode(q, k_cache, v_cache, lengths, sink=None, *, kind="ring", capacity=Non
                                 _ptr(ws), nbytes, _stream(stream))
     _check("mimo_attn_decode", st)
     return out, lse
+
+
+def prefill_chunk(q, k, v, sink=None, *, pos_offset, k_prefix_rotated=True, window=0,
+                  rope_theta=1e4, rot_dims=64, softmax_scale=0.0, out=None, lse=None,
+                  want_lse=True, stream=None):
+    """mimo_attn_prefill_chunk. q [B,n,Hq,192] (the chunk); k, v [B,pos_offset+n,Hkv,·] (every
+    key position; prefix K rotated when k_prefix_rotated). Returns (out [B,n,Hq,128],
+    lse [B,Hq,n])."""
+    _need(q, "q", torch.bfloat16, 4)
+    _need(k, "k", torch.bfloat16, 4)
+    _need(v, "v", torch.bfloat16, 4)
+    B, n, hq, dqk = q.shape
+    _, nk, hkv, _ = k.shape
+    if nk != pos_offset + n or v.shape[:3] != (B, nk, hkv):
+        raise ValueError("k / v must hold positions 0 .. pos_offset + n - 1")
+    if sink is not None:
+        _need(sink, "sink", torch.float32, 1)
+    if out is None:
+        out = torch.empty(B, n, hq, v.shape[3], dtype=torch.bfloat16, device=q.device)
+    if lse is None and want_lse:
+        lse = torch.empty(B, hq, n, dtype=torch.float32, device=q.device)
+    shape = make_shape(B, n, hq, hkv, dqk, v.shape[3], softmax_scale)
+    st = lib().mimo_attn_prefill_chunk(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), int(pos_offset),
+                                       1 if k_prefix_rotated else 0, _ptr(sink), int(window),
+                                       float(rope_theta), int(rot_dims), _ptr(out), _ptr(lse),
+                                       _stream(stream))
+    _check("mimo_attn_prefill_chunk", st)
+    return out, lse
+
+
+def cache_append(k_chunk, v_chunk, k_cache, v_cache, *, pos_offset, rope_theta=1e4, rot_dims=64,
+                 kind="ring", capacity=None, stream=None):
+    """mimo_attn_cache_append: writes the chunk's rotated K and its V into the caches in place."""
+    _need(k_chunk, "k_chunk", torch.bfloat16, 4)
+    _need(v_chunk, "v_chunk", torch.bfloat16, 4)
+    _need(k_cache, "k_cache", torch.bfloat16, 4)
+    _need(v_cache, "v_cache", torch.bfloat16, 4)
+    B, n, hkv, dqk = k_chunk.shape
+    stride = k_cache.shape[1]
+    cap = stride if capacity is None else int(capacity)
+    kind_id = {"ring": MIMO_CACHE_RING, "linear": MIMO_CACHE_LINEAR}[kind]
+    shape = make_shape(B, n, hkv, hkv, dqk, v_chunk.shape[3])
+    st = lib().mimo_attn_cache_append(ctypes.byref(shape), _ptr(k_chunk), _ptr(v_chunk), int(pos_offset),
+                                      float(rope_theta), int(rot_dims), kind_id, _ptr(k_cache),
+                                      _ptr(v_cache), cap, stride, _stream(stream))
+    _check("mimo_attn_cache_append", st)
+    return k_cache, v_cache
 
 
 def decode_mq(q, k_cache, v_cache, lengths, sink=None, *, kind="ring", window=128, capacity=None,

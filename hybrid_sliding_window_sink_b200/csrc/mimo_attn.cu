@@ -131,9 +131,10 @@ mimo_status launch_prefill(const mimo_shape* s, const void* q, const void* k, co
   using C = mimo::PfCfg<G, BN, NKS>;
   CUtensorMap tq, tk, tv;
   const uint64_t n = static_cast<uint64_t>(s->seqlen), B = static_cast<uint64_t>(s->batch);
+  const uint64_t nk = static_cast<uint64_t>(prm.nk);   // keys: n, or prefix + chunk
   if (!make_tmap(&tq, q, mimo::kDQK, s->n_q_heads, n, B, G, C::P) ||
-      !make_tmap(&tk, k, mimo::kDQK, s->n_kv_heads, n, B, 1, BN) ||
-      !make_tmap(&tv, v, mimo::kDV, s->n_kv_heads, n, B, 1, BN))
+      !make_tmap(&tk, k, mimo::kDQK, s->n_kv_heads, nk, B, 1, BN) ||
+      !make_tmap(&tv, v, mimo::kDV, s->n_kv_heads, nk, B, 1, BN))
     return MIMO_ERR_CUDA;
   auto kern = mimo::prefill_kernel<G, BN, NKS>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess) {
@@ -210,6 +211,16 @@ mimo_status prefill_group(const mimo_shape* s, const void* q, const void* k, con
     if (!swa && prm.rot_dims <= 64) return launch_prefill_ga<G>(s, q, k, v, prm, sms, st);
   }
   // one 144-key tile covers the whole window of a row block when P + W - 1 <= 144
+  if (swa && P + prm.window - 1 <= 144) return launch_prefill<G, 144, 1>(s, q, k, v, prm, sms, st);
+  return launch_prefill<G, 128, 2>(s, q, k, v, prm, sms, st);
+}
+
+// Chunked prefill: always the generic kernel (positions offset, keys from a prefix + chunk).
+template <int G>
+mimo_status prefill_chunk_group(const mimo_shape* s, const void* q, const void* k, const void* v,
+                                const PrefillParams& prm, int sms, cudaStream_t st) {
+  constexpr int P = 128 / G;
+  const bool swa = prm.window > 0 && prm.window < prm.nk;
   if (swa && P + prm.window - 1 <= 144) return launch_prefill<G, 144, 1>(s, q, k, v, prm, sms, st);
   return launch_prefill<G, 128, 2>(s, q, k, v, prm, sms, st);
 }
@@ -441,6 +452,9 @@ mimo_status mimo_attn_prefill(const mimo_shape* s, const void* q, const void* k,
   prm.rot_dims = rot_dims;
   prm.rope_theta = static_cast<double>(rope_theta);
   prm.scale_log2 = scale_log2_of(s);
+  prm.q_off = 0;
+  prm.nk = s->seqlen;
+  prm.krot_from = 0;
   prm.err = device_error_ptr(dev);
   if (!prm.err) return MIMO_ERR_CUDA;
 #ifdef MIMO_TRACE
@@ -455,6 +469,91 @@ mimo_status mimo_attn_prefill(const mimo_shape* s, const void* q, const void* k,
     case 8: return prefill_group<8>(s, q, k, v, prm, sms, st);
     default: return prefill_group<16>(s, q, k, v, prm, sms, st);
   }
+}
+
+mimo_status mimo_attn_prefill_chunk(const mimo_shape* s, const void* q, const void* k, const void* v,
+                                    int pos_offset, int k_prefix_rotated, const float* sink,
+                                    int window, float rope_theta, int rot_dims, void* out,
+                                    float* lse, void* stream) {
+  mimo_status e = check_heads(s);
+  if (e != MIMO_OK) return e;
+  if (!q || !k || !v || !out) return MIMO_ERR_NULL;
+  if (s->seqlen < 1 || pos_offset < 0) return MIMO_ERR_SHAPE;
+  if (static_cast<long long>(pos_offset) + s->seqlen > 0x7fffffffLL) return MIMO_ERR_UNSUPPORTED;
+  if (rot_dims < 0 || rot_dims > mimo::kDQK) return MIMO_ERR_SHAPE;
+  if (rot_dims % 16) return MIMO_ERR_UNSUPPORTED;
+  if (rot_dims > 0 && !(rope_theta > 0.f && std::isfinite(rope_theta))) return MIMO_ERR_SHAPE;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) ||
+      (sink && !aligned(sink, 4)) || (lse && !aligned(lse, 4)))
+    return MIMO_ERR_ALIGN;
+  const int dev = current_device();
+  if (dev < 0) return MIMO_ERR_CUDA;
+  PrefillParams prm{};
+  prm.sink = sink;
+  prm.out = static_cast<__nv_bfloat16*>(out);
+  prm.lse = lse;
+  prm.B = s->batch;
+  prm.n = s->seqlen;
+  prm.Hq = s->n_q_heads;
+  prm.Hkv = s->n_kv_heads;
+  prm.window = window;
+  prm.rot_dims = rot_dims;
+  prm.rope_theta = static_cast<double>(rope_theta);
+  prm.scale_log2 = scale_log2_of(s);
+  prm.q_off = pos_offset;
+  prm.nk = pos_offset + s->seqlen;
+  prm.krot_from = k_prefix_rotated ? pos_offset : 0;
+  prm.err = device_error_ptr(dev);
+  if (!prm.err) return MIMO_ERR_CUDA;
+  const int sms = sm_count_for(dev);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  switch (s->n_q_heads / s->n_kv_heads) {
+    case 1: return prefill_chunk_group<1>(s, q, k, v, prm, sms, st);
+    case 2: return prefill_chunk_group<2>(s, q, k, v, prm, sms, st);
+    case 4: return prefill_chunk_group<4>(s, q, k, v, prm, sms, st);
+    case 8: return prefill_chunk_group<8>(s, q, k, v, prm, sms, st);
+    default: return prefill_chunk_group<16>(s, q, k, v, prm, sms, st);
+  }
+}
+
+mimo_status mimo_attn_cache_append(const mimo_shape* s, const void* k_chunk, const void* v_chunk,
+                                   int pos_offset, float rope_theta, int rot_dims, int cache_kind,
+                                   void* k_cache, void* v_cache, int cache_capacity,
+                                   long long seq_stride_tokens, void* stream) {
+  mimo_status e = check_heads(s);
+  if (e != MIMO_OK) return e;
+  if (!k_chunk || !v_chunk || !k_cache || !v_cache) return MIMO_ERR_NULL;
+  if (cache_kind != MIMO_CACHE_RING && cache_kind != MIMO_CACHE_LINEAR) return MIMO_ERR_SHAPE;
+  if (s->seqlen < 1 || pos_offset < 0 || cache_capacity < 1 || seq_stride_tokens < cache_capacity)
+    return MIMO_ERR_SHAPE;
+  if (cache_kind == MIMO_CACHE_LINEAR && static_cast<long long>(pos_offset) + s->seqlen > cache_capacity)
+    return MIMO_ERR_SHAPE;
+  if (static_cast<long long>(pos_offset) + s->seqlen > 0x7fffffffLL) return MIMO_ERR_UNSUPPORTED;
+  if (rot_dims < 0 || rot_dims > mimo::kDQK) return MIMO_ERR_SHAPE;
+  if (rot_dims % 16) return MIMO_ERR_UNSUPPORTED;
+  if (rot_dims > 0 && !(rope_theta > 0.f && std::isfinite(rope_theta))) return MIMO_ERR_SHAPE;
+  if (!aligned(k_chunk, 16) || !aligned(v_chunk, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16))
+    return MIMO_ERR_ALIGN;
+  const int dev = current_device();
+  if (dev < 0) return MIMO_ERR_CUDA;
+  mimo::CacheAppendParams prm{};
+  prm.k = static_cast<const __nv_bfloat16*>(k_chunk);
+  prm.v = static_cast<const __nv_bfloat16*>(v_chunk);
+  prm.kc = static_cast<__nv_bfloat16*>(k_cache);
+  prm.vc = static_cast<__nv_bfloat16*>(v_cache);
+  prm.stride = seq_stride_tokens;
+  prm.B = s->batch;
+  prm.n = s->seqlen;
+  prm.Hkv = s->n_kv_heads;
+  prm.off = pos_offset;
+  prm.rot = rot_dims;
+  prm.ring = cache_kind == MIMO_CACHE_RING;
+  prm.cap = cache_capacity;
+  prm.theta = static_cast<double>(rope_theta);
+  const long long items = static_cast<long long>(s->batch) * s->seqlen * s->n_kv_heads * 40;
+  const long long blocks = std::min<long long>((items + 255) / 256, 4LL * sm_count_for(dev));
+  mimo::cache_append_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(prm);
+  return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ERR_CUDA;
 }
 
 mimo_status mimo_attn_decode(const mimo_shape* s, const void* q, const void* k_cache,

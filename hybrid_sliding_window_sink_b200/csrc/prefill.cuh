@@ -46,6 +46,10 @@ struct PrefillParams {
   double rope_theta;
   float scale_log2;        // softmax scale * log2(e)
   int n_qtiles, num_work;
+  // chunked prefill (generic kernel only): query row i sits at position q_off + i; keys
+  // cover positions 0 .. nk-1; key rows at positions < krot_from are stored rotated.
+  // Whole-sequence prefill: q_off = 0, nk = n, krot_from = 0.
+  int q_off, nk, krot_from;
   unsigned* err;
   unsigned long long* trace;   // debug timestamps (builds with -DMIMO_TRACE only), else null
 };
@@ -130,6 +134,18 @@ __device__ __forceinline__ void rope_row(uint32_t base, int chunk_bytes, int row
   }
 }
 
+// A key row stored already rotated (a cached prefix): its first `rot` dims only change
+// format, bf16 -> f16, to match the f16 MMA k-steps over the rotated dims.
+__device__ __forceinline__ void f16_row(uint32_t base, int chunk_bytes, int row, int rot) {
+  for (int u = 0; u < (rot >> 3); ++u) {
+    const uint32_t a = base + (u >> 3) * chunk_bytes + row * 128 + (((u & 7) ^ (row & 7)) << 4);
+    uint32_t x[4];
+    ld_shared_v4(a, x[0], x[1], x[2], x[3]);
+    st_shared_v4(a, bf16x2_to_f16x2(x[0]), bf16x2_to_f16x2(x[1]), bf16x2_to_f16x2(x[2]),
+                 bf16x2_to_f16x2(x[3]));
+  }
+}
+
 template <int G, int BN, int NKS>
 __global__ void __launch_bounds__(kPfThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -179,7 +195,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
 
-  const bool swa = p.window > 0 && p.window < p.n;
+  const bool swa = p.window > 0 && p.window < p.nk;
   const int BG = p.B * p.Hkv;
   auto work_of = [&](int w, int& b, int& g, int& qt) {
     if (swa) {   // neighbouring CTAs take neighbouring row blocks: K/V windows overlap in L2
@@ -195,8 +211,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
   };
   auto kv_range = [&](int qt, int& lo, int& ntiles) {
-    const int p0 = qt * C::P;
-    const int hi = min(p0 + C::P - 1, p.n - 1);
+    const int p0 = p.q_off + qt * C::P;                  // absolute position of the block
+    const int hi = min(p0 + C::P - 1, p.q_off + p.n - 1);
     lo = swa ? max(0, p0 - p.window + 1) : 0;
     ntiles = (hi - lo + BN) / BN;
   };
@@ -310,7 +326,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         const uint32_t sK = sK0 + ks * C::K_BYTES;
         for (int t = ctid; t < BN; t += 128) {
           const int pos = key0 + t;
-          if (pos < p.n) rope_row(sK, C::K_CHUNK, t, pos, p.rot_dims, s_invf);
+          if (pos >= p.krot_from && pos < p.nk) rope_row(sK, C::K_CHUNK, t, pos, p.rot_dims, s_invf);
+          else if (pos >= 0 && pos < p.krot_from) f16_row(sK, C::K_CHUNK, t, p.rot_dims);
         }
         fence_proxy_async_smem();
       }
@@ -322,9 +339,10 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       int b, g, qt, lo, T;
       work_of(w, b, g, qt);
       kv_range(qt, lo, T);
-      const int pos = qt * C::P + r / G;
+      const int qi = qt * C::P + r / G;                  // query row within the call
+      const int pos = p.q_off + qi;                      // its position
       const int h = g * G + (r % G);
-      const bool row_ok = pos < p.n;
+      const bool row_ok = qi < p.n;
       const int klo = swa ? pos - p.window + 1 : 0;   // valid keys: [klo, pos]
 
       if (!wait_all(bar(kBarQFull), it_q & 1)) { ok = false; break; }
@@ -419,7 +437,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       if (!wait_all(bar(kBarPVDone), (it_kv + T - 1) & 1)) { ok = false; break; }
       tc_fence_after();
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
-      __nv_bfloat16* orow = p.out + ((static_cast<long long>(b) * p.n + pos) * p.Hq + h) * 128;
+      __nv_bfloat16* orow = p.out + ((static_cast<long long>(b) * p.n + qi) * p.Hq + h) * 128;
 #pragma unroll 1
       for (int cb = 0; cb < 8; ++cb) {
         uint32_t v[16];
@@ -436,7 +454,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         }
       }
       if (row_ok && p.lse)
-        p.lse[(static_cast<long long>(b) * p.Hq + h) * p.n + pos] =
+        p.lse[(static_cast<long long>(b) * p.Hq + h) * p.n + qi] =
             l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
       tc_fence_before();
       it_kv += T;
@@ -448,6 +466,74 @@ __global__ void __launch_bounds__(kPfThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+}
+
+// Appends a chunk of n tokens (positions off .. off+n-1) to a KV cache: K rotated at its
+// position (rotate-half pairing over the first rot dims, angles reduced in double precision)
+// and rounded to bf16, V copied. One thread per 16-byte unit of an output row; slot =
+// p mod cap (ring, only the chunk's last cap tokens) or p (linear).
+struct CacheAppendParams {
+  const __nv_bfloat16* k;     // [B, n, Hkv, 192]
+  const __nv_bfloat16* v;     // [B, n, Hkv, 128]
+  __nv_bfloat16* kc;          // [B, stride, Hkv, 192]
+  __nv_bfloat16* vc;          // [B, stride, Hkv, 128]
+  long long stride;
+  int B, n, Hkv, off, rot, ring, cap;
+  double theta;
+};
+
+__global__ void __launch_bounds__(256) cache_append_kernel(const CacheAppendParams p) {
+  constexpr int kUnits = 24 + 16;                       // K units, then V units, per row
+  const long long total = static_cast<long long>(p.B) * p.n * p.Hkv * kUnits;
+  const int first = p.ring && p.n > p.cap ? p.n - p.cap : 0;   // older chunk tokens are overwritten
+  const int half = p.rot >> 1;
+  for (long long it = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; it < total;
+       it += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int u = static_cast<int>(it % kUnits);
+    const long long row = it / kUnits;                  // (b, i, g)
+    const int g = static_cast<int>(row % p.Hkv);
+    const long long bi = row / p.Hkv;
+    const int i = static_cast<int>(bi % p.n), b = static_cast<int>(bi / p.n);
+    if (i < first) continue;
+    const int pos = p.off + i;
+    const long long slot = p.ring ? pos % p.cap : pos;
+    const long long dst_row = (static_cast<long long>(b) * p.stride + slot) * p.Hkv + g;
+    if (u >= 24) {                                      // V: copy 16 bytes
+      const int vu = u - 24;
+      *reinterpret_cast<uint4*>(p.vc + dst_row * 128 + vu * 8) =
+          *reinterpret_cast<const uint4*>(p.v + row * 128 + vu * 8);
+      continue;
+    }
+    const __nv_bfloat16* src = p.k + row * 192;
+    uint4 x = *reinterpret_cast<const uint4*>(src + u * 8);
+    if (u * 8 < p.rot) {
+      // dims d = 8u .. 8u+7: partner dims d -+ half
+      const bool first_half = u * 8 < half;
+      const int pu = first_half ? u + (half >> 3) : u - (half >> 3);
+      const uint4 y = *reinterpret_cast<const uint4*>(src + pu * 8);
+      const uint32_t xs[4] = {x.x, x.y, x.z, x.w}, ys[4] = {y.x, y.y, y.z, y.w};
+      uint32_t out[4];
+#pragma unroll
+      for (int e2 = 0; e2 < 4; ++e2) {
+        float r[2];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const int d = u * 8 + e2 * 2 + hh;
+          const int k = first_half ? d : d - half;
+          const double ang = static_cast<double>(pos) * pow(p.theta, -2.0 * k / static_cast<double>(p.rot));
+          const double nrev = rint(ang * 0.15915494309189535);
+          float sn, cs;
+          sincosf(static_cast<float>(fma(-nrev, 6.283185307179586, ang)), &sn, &cs);
+          const float a = hh ? bf16_hi(xs[e2]) : bf16_lo(xs[e2]);
+          const float bp = hh ? bf16_hi(ys[e2]) : bf16_lo(ys[e2]);
+          r[hh] = first_half ? a * cs - bp * sn : a * cs + bp * sn;
+        }
+        out[e2] = pack_bf16(r[0], r[1]);
+      }
+      x = make_uint4(out[0], out[1], out[2], out[3]);
+    }
+    *reinterpret_cast<uint4*>(p.kc + dst_row * 192 + u * 8) = x;
   }
 }
 

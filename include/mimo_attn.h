@@ -153,6 +153,46 @@ mimo_status mimo_attn_sparse(const mimo_shape* shape, const void* q, const void*
                              void* stream);
 
 /*
+ * Chunked prefill over a KV prefix (youngju.dev "mimo-v25-inference-optimization", serving
+ * section: long prompts are prefilled in chunks). A chunk of n = shape->seqlen query tokens
+ * at positions pos_offset .. pos_offset + n - 1 attends the keys of positions
+ * 0 .. pos_offset + n - 1, exactly as those rows of mimo_attn_prefill over the whole sequence.
+ *
+ *  q    [B, n, Hq, 192] bf16 device, un-rotated (rotated here at their positions)
+ *  k, v [B, pos_offset + n, Hkv, 192 | 128] bf16 device: every key position. The chunk's
+ *       rows (positions >= pos_offset) are un-rotated; the prefix rows are taken as stored
+ *       when k_prefix_rotated != 0 (as a KV cache holds them) and rotated here otherwise
+ *  pos_offset >= 0; sink, window (<= 0 or >= pos_offset + n: full causal), rope_theta,
+ *       rot_dims: as mimo_attn_prefill
+ *  out  [B, n, Hq, 128] bf16 device; lse [B, Hq, n] fp32 device or NULL
+ *
+ * Runs on the generic prefill kernel (not the SWA ring or GA pair kernels). Errors as
+ * mimo_attn_prefill; MIMO_ERR_SHAPE also for pos_offset < 0.
+ */
+mimo_status mimo_attn_prefill_chunk(const mimo_shape* shape, const void* q, const void* k,
+                                    const void* v, int pos_offset, int k_prefix_rotated,
+                                    const float* sink, int window, float rope_theta, int rot_dims,
+                                    void* out, float* lse, void* stream);
+
+/*
+ * Writes a chunk of n = shape->seqlen tokens (positions pos_offset .. pos_offset + n - 1) into
+ * a KV cache, as the decode calls read it: K rotated at its position (first rot_dims dims,
+ * rotate-half pairing, theta rope_theta) and rounded to bf16, V copied; token p goes to slot
+ * p mod cache_capacity (MIMO_CACHE_RING, only the chunk's last cache_capacity tokens are
+ * written) or slot p (MIMO_CACHE_LINEAR, pos_offset + n <= cache_capacity).
+ *
+ *  k_chunk [B, n, Hkv, 192], v_chunk [B, n, Hkv, 128] bf16 device (un-rotated K)
+ *  k_cache [B, seq_stride_tokens, Hkv, 192], v_cache [.., 128] bf16 device, written in place
+ *
+ * Errors: MIMO_ERR_NULL, MIMO_ERR_SHAPE (bad kind, sizes, a linear cache too small),
+ * MIMO_ERR_UNSUPPORTED (rot_dims not a multiple of 16), MIMO_ERR_ALIGN, MIMO_ERR_CUDA.
+ */
+mimo_status mimo_attn_cache_append(const mimo_shape* shape, const void* k_chunk,
+                                   const void* v_chunk, int pos_offset, float rope_theta,
+                                   int rot_dims, int cache_kind, void* k_cache, void* v_cache,
+                                   int cache_capacity, long long seq_stride_tokens, void* stream);
+
+/*
  * Multi-query decode: MTP draft verification (syt-nju.github.io "mimo-mtp-swa-not-mla",
  * MTP section: the main model checks the draft tokens in one forward pass). The q_len
  * newest tokens of each sequence, at positions L_b - q_len .. L_b - 1 and already written

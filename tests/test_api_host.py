@@ -157,3 +157,23 @@ def test_decode_mq_workspace_plans(L):
                                                 128) == 0
     assert L.mimo_attn_decode_mq_workspace_size(ctypes.byref(lin), _lib.MIMO_CACHE_LINEAR, 4096, 8,
                                                 0) == 0
+
+
+def test_prefill_chunk_and_append_reject_before_launch(L):
+    s = _shape(hq=64, hkv=8, seqlen=100)
+    chunk = lambda **kw: L.mimo_attn_prefill_chunk(  # noqa: E731
+        ctypes.byref(s), kw.get("q", GOOD), GOOD, GOOD, kw.get("off", 10), 1, None, 128,
+        kw.get("theta", 1e4), kw.get("rot", 64), GOOD, None, None)
+    assert chunk(off=-1) == 2
+    assert chunk(q=None) == 1
+    assert chunk(rot=24) == 3
+    assert chunk(theta=0.0) == 2
+    assert chunk(q=P(0x10004)) == 4
+    app = lambda **kw: L.mimo_attn_cache_append(  # noqa: E731
+        ctypes.byref(s), GOOD, GOOD, kw.get("off", 0), 1e4, 64, kw.get("kind", _lib.MIMO_CACHE_LINEAR),
+        kw.get("kc", GOOD), GOOD, kw.get("cap", 1000), kw.get("stride", 1000), None)
+    assert app(off=950) == 2                          # linear cache too small for the chunk
+    assert app(kind=5) == 2
+    assert app(kc=None) == 1
+    assert app(stride=999) == 2
+    assert app(kc=P(0x10008)) == 4
