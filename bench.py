@@ -238,6 +238,45 @@ def bench_prefill(case, steps, warmup, peaks, tag, dev, stream):
     return res
 
 
+def bench_chunk_prefill(steps, warmup, peaks, tag, dev, stream, chunk=16384, prefix=16384):
+    """Chunked prefill (16K chunk after a 16K prefix held rotated, as a cache holds it), B=1,
+    on an SWA layer (64Q/8KV, W=128, HBM-bound) and a GA layer (64Q/4KV, tensor-bound)."""
+    from hybrid_sliding_window_sink_b200 import _lib
+    res = {}
+    nk = prefix + chunk
+    for name, hq, hkv, window, theta in (("swa", 64, 8, wl.SWA_WINDOW, wl.SWA_THETA),
+                                         ("ga", 64, 4, 0, wl.GA_THETA)):
+        inp = wl.prefill_inputs(1, nk, hq, hkv, seed=1700, device=dev, k_scale=0.5 if window == 0 else 1.0)
+        q = inp["q"][:, prefix:].contiguous()
+        out = torch.empty(1, chunk, hq, wl.DV, dtype=torch.bfloat16, device=dev)
+        lse = torch.empty(1, hq, chunk, dtype=torch.float32, device=dev)
+
+        def step():
+            _lib.prefill_chunk(q, inp["k"], inp["v"], inp["sink"], pos_offset=prefix, k_prefix_rotated=True,
+                               window=window, rope_theta=theta, rot_dims=wl.ROT_DIMS, out=out, lse=lse,
+                               stream=stream)
+
+        n_steps = steps if window > 0 else max(3, steps // 20)
+        ms = timed(step, n_steps, warmup, stream) / n_steps
+        if window > 0:
+            pairs = sum(min(window, prefix + i + 1) for i in range(chunk))
+            bytes_ = (chunk * hq * wl.DQK * 2 + (chunk + window - 1) * hkv * (wl.DQK + wl.DV) * 2
+                      + chunk * hq * wl.DV * 2 + hq * chunk * 4)
+        else:
+            pairs = chunk * prefix + chunk * (chunk + 1) // 2
+            bytes_ = chunk * hq * wl.DQK * 2 + nk * hkv * (wl.DQK + wl.DV) * 2 + chunk * hq * (wl.DV * 2 + 4)
+        flops = 2.0 * (wl.DQK + wl.DV) * pairs * hq
+        res[name] = {"ms": round(ms, 4), "tflops": round(flops / (ms * 1e-3) / 1e12, 2),
+                     "roofline": (roofline_hbm(bytes_, ms, peaks, tag) if window > 0 else
+                                  roofline_tensor(flops, ms, peaks["bf16_tflops"], tag)),
+                     "device_error": _lib.last_device_error()}
+        del inp, q, out, lse
+        torch.cuda.empty_cache()
+    res["workload"] = f"chunked prefill, {chunk}-token chunk after a {prefix}-token prefix (rotated), B=1"
+    res["kernel"] = "generic tcgen05 prefill kernel (one compute warpgroup)"
+    return res
+
+
 def e2e_prefill(case, steps, dev, stream):
     """Same metric through the public call with host buffers: pinned H2D of the step's
     inputs, the kernel, D2H of the outputs, all inside the timed region."""
@@ -650,6 +689,10 @@ def main():
             torch.cuda.empty_cache()
         except Exception as e:  # report, do not hide
             wls["ga_prefill"] = {"error": repr(e)}
+        try:
+            wls["chunk_prefill"] = bench_chunk_prefill(max(3, ksteps), 3, peaks, tag, dev, stream)
+        except Exception as e:
+            wls["chunk_prefill"] = {"error": repr(e)}
         try:
             wls["hybrid_decode_step"] = bench_decode_step(max(3, ksteps), 3, peaks, tag, dev, stream)
             wls["hybrid_decode_step"]["workload"] = "hybrid decode step, 48 layers, B=64"

@@ -15,6 +15,8 @@ Cases:
                         tokens (all full), 64 Q / 4 KV heads
   fp8_linear_b64_l16k   GA decode over an FP8 (E4M3 + per-row scale) linear cache, B=64, 16384
                         tokens (all full), 64 Q / 4 KV heads
+  chunk_ga_c8192_p8192  GA chunked prefill: 8192-token chunk after an 8192-token rotated prefix,
+                        64 Q / 4 KV heads (generic prefill kernel)
 Prints the mean time per call over --reps calls (after two warm-up calls).
 """
 
@@ -73,6 +75,11 @@ def _case(name, dev):
                          dtype=torch.uint8, device=dev)
         return lambda: _lib.decode_fp8(d["q"], d["k8"], d["v8"], d["k_scale"], d["v_scale"],
                                        d["lengths"], d["sink"], kind="linear", workspace=ws)
+    if name == "chunk_ga_c8192_p8192":
+        inp = wl.prefill_inputs(1, 16384, 64, 4, seed=12, device=dev, k_scale=0.5)
+        q = inp["q"][:, 8192:].contiguous()
+        return lambda: _lib.prefill_chunk(q, inp["k"], inp["v"], inp["sink"], pos_offset=8192,
+                                          k_prefix_rotated=True, window=0, rope_theta=1e7, rot_dims=64)
     raise SystemExit(f"unknown case {name}")
 
 
