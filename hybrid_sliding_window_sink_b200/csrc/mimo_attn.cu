@@ -182,9 +182,10 @@ mimo_status launch_prefill_ga(const mimo_shape* s, const void* q, const void* k,
   using L = mimo::GaLayout<G>;
   CUtensorMap tq, tk, tv;
   const uint64_t n = static_cast<uint64_t>(s->seqlen), B = static_cast<uint64_t>(s->batch);
+  const uint64_t nk = static_cast<uint64_t>(prm.nk);   // keys: n, or prefix + chunk
   if (!make_tmap(&tq, q, mimo::kDQK, s->n_q_heads, n, B, G, L::P) ||
-      !make_tmap(&tk, k, mimo::kDQK, s->n_kv_heads, n, B, 1, mimo::kGaBN) ||
-      !make_tmap(&tv, v, mimo::kDV, s->n_kv_heads, n, B, 1, mimo::kGaBN))
+      !make_tmap(&tk, k, mimo::kDQK, s->n_kv_heads, nk, B, 1, mimo::kGaBN) ||
+      !make_tmap(&tv, v, mimo::kDV, s->n_kv_heads, nk, B, 1, mimo::kGaBN))
     return MIMO_ERR_CUDA;
   auto kern = mimo::prefill_ga_kernel<G>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM) != cudaSuccess) {
@@ -215,12 +216,16 @@ mimo_status prefill_group(const mimo_shape* s, const void* q, const void* k, con
   return launch_prefill<G, 128, 2>(s, q, k, v, prm, sms, st);
 }
 
-// Chunked prefill: always the generic kernel (positions offset, keys from a prefix + chunk).
+// Chunked prefill: GA layers with 8 or 16 query heads per KV head on the pair kernel, every
+// other shape on the generic kernel (query positions offset, keys from a prefix + the chunk).
 template <int G>
 mimo_status prefill_chunk_group(const mimo_shape* s, const void* q, const void* k, const void* v,
                                 const PrefillParams& prm, int sms, cudaStream_t st) {
   constexpr int P = 128 / G;
   const bool swa = prm.window > 0 && prm.window < prm.nk;
+  if constexpr (G == 8 || G == 16) {   // full causal prefix: the pair kernel
+    if (!swa && prm.rot_dims <= 64) return launch_prefill_ga<G>(s, q, k, v, prm, sms, st);
+  }
   if (swa && P + prm.window - 1 <= 144) return launch_prefill<G, 144, 1>(s, q, k, v, prm, sms, st);
   return launch_prefill<G, 128, 2>(s, q, k, v, prm, sms, st);
 }

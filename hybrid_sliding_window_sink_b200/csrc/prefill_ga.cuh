@@ -168,8 +168,8 @@ __global__ void __launch_bounds__(kGaThreads, 1)
     const int pi = npairs - 1 - w / BG;
     b = bg / p.Hkv;
     g = bg - b * p.Hkv;
-    p0 = pi * 2 * P;
-    const int hi = min(p0 + 2 * P - 1, p.n - 1);
+    p0 = pi * 2 * P;                               // first query row of block A in the call
+    const int hi = p.q_off + min(p0 + 2 * P - 1, p.n - 1);   // last position of the item
     ntiles = hi / kGaBN + 1;
   };
 
@@ -338,8 +338,9 @@ __global__ void __launch_bounds__(kGaThreads, 1)
       if (!wait_all(bar(kGaQFull), it & 1)) { ok = false; break; }
       if (half > 0) {
         for (int blk = 0; blk < 2; ++blk) {
-          const int pos = p0 + blk * P + ctid / G;
-          if (pos < p.n) rope_row(sQ + blk * L::Q_BLOCK, L::Q_CHUNK, ctid, pos, p.rot_dims, s_invf);
+          const int qi = p0 + blk * P + ctid / G;
+          if (qi < p.n)
+            rope_row(sQ + blk * L::Q_BLOCK, L::Q_CHUNK, ctid, p.q_off + qi, p.rot_dims, s_invf);
         }
         fence_proxy_async_smem();
       }
@@ -365,7 +366,17 @@ __global__ void __launch_bounds__(kGaThreads, 1)
           }
           if (!wait_all(bar(kGaBase + tb), (gt >> 2) & 1)) { ok = false; break; }
           if (!wait_all(bar(kGaKFull + ks), (gt >> 1) & 1)) { ok = false; break; }
-          if (kt0 + ctid < p.n) {
+          if (kt0 + ctid < p.nk && kt0 + ctid < p.krot_from) {
+            // a prefix row stored rotated (from a KV cache): only bf16 -> f16 for the f16
+            // MMA k-steps over the rotated dims
+            uint8_t* row = smem + L::OFF_K + ks * L::K_TILE + ctid * 128;
+            for (int u = 0; u < (half >> 2); ++u) {
+              uint4* px = reinterpret_cast<uint4*>(row + ((u ^ (ctid & 7)) << 4));
+              const uint4 xv = *px;
+              *px = make_uint4(bf16x2_to_f16x2(xv.x), bf16x2_to_f16x2(xv.y), bf16x2_to_f16x2(xv.z),
+                               bf16x2_to_f16x2(xv.w));
+            }
+          } else if (kt0 + ctid < p.nk) {
             // rotate row ctid of the tile: angle (kt0 + t) w_k from base_k and own_k
             uint8_t* row = smem + L::OFF_K + ks * L::K_TILE + ctid * 128;
             const int nun = half >> 3;
@@ -420,10 +431,11 @@ __global__ void __launch_bounds__(kGaThreads, 1)
     for (int rd = 0, w = work_of(0); w < p.num_work && ok; w = work_of(++rd)) {
       int b, g, p0, T;
       item_of(w, b, g, p0, T);
-      const int pmin = p0 + grp * P;              // first position of this row block
+      const int pmin = p.q_off + p0 + grp * P;    // first position of this row block
       const int pos = pmin + r / G;
+      const int qi = pos - p.q_off;               // query row within the call
       const int hq = g * G + (r % G);
-      const bool row_ok = pos < p.n;
+      const bool row_ok = qi < p.n;
       const float sink2 = p.sink ? p.sink[hq] * kLog2e : -INFINITY;
       float m = sink2;                             // reference max (log2 units)
       float l = p.sink ? 1.f : 0.f;
@@ -528,7 +540,7 @@ __global__ void __launch_bounds__(kGaThreads, 1)
       if (!wait_all(bar(kGaPVDone + grp), (gt - 1) & 1)) { ok = false; break; }
       tc_fence_after();
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
-      __nv_bfloat16* orow = p.out + ((static_cast<long long>(b) * p.n + pos) * p.Hq + hq) * 128;
+      __nv_bfloat16* orow = p.out + ((static_cast<long long>(b) * p.n + qi) * p.Hq + hq) * 128;
 #pragma unroll 1
       for (int c = 0; c < 8; c += 2) {
         uint32_t v0[16], v1[16];
@@ -550,7 +562,7 @@ __global__ void __launch_bounds__(kGaThreads, 1)
         }
       }
       if (row_ok && p.lse)
-        p.lse[(static_cast<long long>(b) * p.Hq + hq) * p.n + pos] =
+        p.lse[(static_cast<long long>(b) * p.Hq + hq) * p.n + qi] =
             l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
       tc_fence_before();
     }
