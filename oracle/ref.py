@@ -47,6 +47,11 @@ Readings where the pages are silent (each also listed in the design notes):
   keys may come from a KV cache (already rotated) or un-rotated; the chunk's own keys are
   un-rotated. Appending a chunk to a cache stores its rotated K and its V at slot
   p mod capacity (ring) or p (linear) for each of its positions p.
+* Token selection (aideepthink.cn §二.2 / §四.3: token-level, reused from the preceding
+  full-attention layer, no separately trained retrieval module; the scoring rule itself
+  is not given): for a sequence and KV head, every token outside the recent window is
+  scored by its largest attention logit over the group's query heads; the n_sel best
+  are kept (equal scores: lower index first) and returned in increasing order.
 * FP8 KV cache (the pages size their KV caches in FP8 but give no scaling scheme):
   K and V bytes are OCP FP8 E4M3 (bias 7, no infinities, S.1111.111 is NaN), each
   (token, KV head) row carries one fp32 scale per tensor, and the cached value is
@@ -73,6 +78,7 @@ __all__ = [
     "sparse_key_set",
     "prefill_chunk",
     "cache_append",
+    "select_tokens",
     "e4m3_to_float",
     "dequant_fp8",
     "decode_fp8",
@@ -414,6 +420,33 @@ def combine_partials(parts, sink):
         L += math.exp(float(sink) - M)
     o = sum(oc * math.exp(m - M) for m, _, oc in parts) / L
     return o, M + math.log(L)
+
+
+# --------------------------------------------------------------------------
+# Token selection for the sparse decode
+# --------------------------------------------------------------------------
+
+def select_tokens(q, k_cache, lengths, recent: int, n_sel: int, scale=None) -> np.ndarray:
+    """sel [B, Hkv, n_sel] int64: per sequence b and KV head g, the n_sel tokens t in
+    [0, L_b - recent) with the largest score max_{h in group g} (q_h . k_t) * scale, equal
+    scores taken in increasing t, listed in increasing t. q: [B, Hq, Dqk] (rotated);
+    k_cache: [B, cap, Hkv, Dqk] linear (rotated K)."""
+    q, kc = _f64(q), _f64(k_cache)
+    B, Hq, D = q.shape
+    Hkv = kc.shape[2]
+    group = Hq // Hkv
+    sc = _scale(scale, D)
+    out = np.zeros((B, Hkv, n_sel), dtype=np.int64)
+    for b in range(B):
+        hi = int(lengths[b]) - recent
+        if hi < n_sel:
+            raise ValueError("fewer candidate tokens than n_sel")
+        for g in range(Hkv):
+            logits = (kc[b, :hi, g, :] @ q[b, g * group:(g + 1) * group, :].T) * sc   # [hi, group]
+            score = logits.max(axis=1)
+            order = sorted(range(hi), key=lambda t: (-score[t], t))
+            out[b, g] = np.sort(np.asarray(order[:n_sel], dtype=np.int64))
+    return out
 
 
 # --------------------------------------------------------------------------

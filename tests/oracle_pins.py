@@ -384,6 +384,54 @@ def check_chunked_prefill_matches_whole(ref):
         np.testing.assert_allclose(l[0], l_pf[0, :, L - 1], rtol=0, atol=1e-11)
 
 
+def check_select_tokens(ref):
+    """Token selection (aideepthink.cn §四.3 key set; scoring rule taken as the largest
+    group logit): against a direct per-token scan, the kept set is exactly the n_sel best
+    (every kept score >= every dropped one), ties go to the lower index, the order is
+    increasing, heads of a group commute, positive scalings of q do not change the choice,
+    and with n_sel = all candidates the sparse decode over the chosen set equals decode over
+    the whole cache."""
+    r = _rng(37)
+    B, Hq, Hkv, D, cap = 2, 8, 2, 16, 60
+    q = r.integers(-2, 3, size=(B, Hq, D)).astype(np.float64)
+    k = r.integers(-2, 3, size=(B, cap, Hkv, D)).astype(np.float64)
+    lengths, recent, n_sel = [60, 45], 8, 10
+    sel = ref.select_tokens(q, k, lengths, recent, n_sel)
+    group = Hq // Hkv
+    for b in range(B):
+        hi = lengths[b] - recent
+        for g in range(Hkv):
+            s = sel[b, g]
+            assert len(s) == n_sel and np.all(np.diff(s) > 0) and s[0] >= 0 and s[-1] < hi
+            score = np.array([max(float(q[b, h] @ k[b, t, g]) for h in range(g * group, (g + 1) * group))
+                              for t in range(hi)])
+            kept = set(s.tolist())
+            dropped = [t for t in range(hi) if t not in kept]
+            assert min(score[list(kept)]) >= max(score[dropped])
+            thr = min(score[list(kept)])
+            # ties at the threshold: the kept ones are the lowest indices among them
+            tied = [t for t in range(hi) if score[t] == thr]
+            n_tied_kept = sum(1 for t in tied if t in kept)
+            assert [t for t in tied if t in kept] == tied[:n_tied_kept]
+    # a constructed tie: equal scores everywhere -> the first n_sel candidates
+    qz = np.zeros((1, 4, D))
+    kz = r.standard_normal((1, 30, 1, D))
+    assert np.array_equal(ref.select_tokens(qz, kz, [30], 5, 7)[0, 0], np.arange(7))
+    # heads of a group commute; positive scaling of q keeps the choice
+    perm = np.arange(Hq).reshape(Hkv, group)[:, ::-1].ravel()
+    assert np.array_equal(ref.select_tokens(q[:, perm], k, lengths, recent, n_sel), sel)
+    assert np.array_equal(ref.select_tokens(q * 3.5, k, lengths, recent, n_sel), sel)
+    # n_sel = every candidate: sparse decode over it is decode over the whole cache
+    v = r.standard_normal((B, cap, Hkv, 8))
+    sink = r.standard_normal(Hq)
+    L = [60, 60]
+    full_sel = ref.select_tokens(q, k, L, recent, 60 - recent)
+    o1, l1 = ref.sparse_decode(q, k, v, L, recent, full_sel, sink)
+    o2, l2 = ref.decode(q, k, v, "linear", L, sink)
+    np.testing.assert_allclose(o1, o2, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(l1, l2, rtol=0, atol=1e-12)
+
+
 def check_e4m3_decoding(ref):
     """OCP FP8 E4M3: every one of the 256 byte patterns decodes as torch.float8_e4m3fn
     does, and the landmarks of the format hold (1.0, the largest 448, the smallest
@@ -520,6 +568,7 @@ ALL_CHECKS = [
     check_decode_matches_prefill,
     check_multi_decode_matches_prefill,
     check_chunked_prefill_matches_whole,
+    check_select_tokens,
     check_sparse_membership,
     check_e4m3_decoding,
     check_fp8_decode_reduces_to_bf16,

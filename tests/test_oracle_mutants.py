@@ -51,6 +51,13 @@ MUTANTS = {
     "appended K left un-rotated": ("            kc[b, slot] = kr[i]\n", "            kc[b, slot] = kn[b, i]\n"),
     "ring append without modulo": ("            slot = p % cap if kind == \"ring\" else p\n",
                                    "            slot = min(p, cap - 1)\n"),
+    "selection keeps the worst": ("            order = sorted(range(hi), key=lambda t: (-score[t], t))\n",
+                                  "            order = sorted(range(hi), key=lambda t: (score[t], t))\n"),
+    "selection ties to the higher index": ("            order = sorted(range(hi), key=lambda t: (-score[t], t))\n",
+                                           "            order = sorted(range(hi), key=lambda t: (-score[t], -t))\n"),
+    "selection by the group's mean logit": ("            score = logits.max(axis=1)\n", "            score = logits.mean(axis=1)\n"),
+    "selection reaches into the window": ("        hi = int(lengths[b]) - recent\n        if hi < n_sel:",
+                                          "        hi = int(lengths[b]) - recent + 1\n        if hi < n_sel:"),
     "e4m3 exponent bias 8": ("np.exp2(e.astype(np.float64) - 7.0)", "np.exp2(e.astype(np.float64) - 8.0)"),
     "e4m3 subnormal scale": ("m / 8.0 * 2.0 ** -6", "m / 8.0 * 2.0 ** -7"),
     "e4m3 without NaN": ("np.where((e == 15) & (m == 7), np.nan, val)", "val"),
