@@ -28,7 +28,7 @@ STATUS = {0: "MIMO_OK", 1: "MIMO_ERR_NULL", 2: "MIMO_ERR_SHAPE", 3: "MIMO_ERR_UN
 EXPORTS = ("mimo_attn_prefill", "mimo_attn_decode", "mimo_attn_sparse", "mimo_attn_sparse_noalloc",
            "mimo_attn_decode_mq", "mimo_attn_decode_mq_workspace_size", "mimo_attn_workspace_size",
            "mimo_attn_decode_fp8", "mimo_attn_sparse_fp8", "mimo_attn_prefill_chunk",
-           "mimo_attn_cache_append",
+           "mimo_attn_cache_append", "mimo_attn_select_tokens", "mimo_attn_select_workspace_size",
            "mimo_attn_check_indices", "mimo_attn_last_device_error", "mimo_status_string",
            "mimo_attn_version")
 
@@ -71,6 +71,9 @@ def lib():
     L.mimo_attn_decode_mq_workspace_size.restype = SZ
     L.mimo_attn_prefill_chunk.argtypes = [SP, P, P, P, I, I, P, I, F, I, P, P, P]
     L.mimo_attn_cache_append.argtypes = [SP, P, P, I, F, I, I, P, P, I, LL, P]
+    L.mimo_attn_select_tokens.argtypes = [SP, P, P, I, LL, P, I, I, P, P, SZ, P]
+    L.mimo_attn_select_workspace_size.argtypes = [SP, I]
+    L.mimo_attn_select_workspace_size.restype = SZ
     L.mimo_attn_decode_fp8.argtypes = [SP, P, P, P, P, P, I, I, LL, P, P, P, P, P, SZ, P]
     L.mimo_attn_sparse_fp8.argtypes = [SP, P, P, P, P, P, I, LL, P, I, P, I, P, P, P, P, SZ, P]
     L.mimo_attn_workspace_size.argtypes = [SP, I, I, I, I, I]
@@ -243,6 +246,28 @@ def cache_append(k_chunk, v_chunk, k_cache, v_cache, *, pos_offset, rope_theta=1
                                       _ptr(v_cache), cap, stride, _stream(stream))
     _check("mimo_attn_cache_append", st)
     return k_cache, v_cache
+
+
+def select_tokens(q, k_cache, lengths, *, recent=128, n_sel=1024, capacity=None, out=None,
+                  workspace=None, stream=None):
+    """mimo_attn_select_tokens. q [B,Hq,192]; linear k_cache [B,stride,Hkv,192] (rotated K);
+    lengths [B] int32. Returns sel_idx [B,Hkv,n_sel] int32 (sorted, as sparse() reads it)."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(k_cache, "k_cache", torch.bfloat16, 4)
+    _need(lengths, "lengths", torch.int32, 1)
+    B, hq, dqk = q.shape
+    _, stride, hkv, _ = k_cache.shape
+    cap = stride if capacity is None else int(capacity)
+    if out is None:
+        out = torch.empty(B, hkv, n_sel, dtype=torch.int32, device=q.device)
+    shape = make_shape(B, 1, hq, hkv, dqk)
+    nbytes = int(lib().mimo_attn_select_workspace_size(ctypes.byref(shape), cap))
+    ws = _workspace(workspace, nbytes, q.device)
+    st = lib().mimo_attn_select_tokens(ctypes.byref(shape), _ptr(q), _ptr(k_cache), cap, stride,
+                                       _ptr(lengths), int(recent), int(n_sel), _ptr(out), _ptr(ws),
+                                       nbytes, _stream(stream))
+    _check("mimo_attn_select_tokens", st)
+    return out
 
 
 def decode_mq(q, k_cache, v_cache, lengths, sink=None, *, kind="ring", window=128, capacity=None,

@@ -15,6 +15,7 @@
 #include "ptx.cuh"
 #include "decode.cuh"
 #include "decode_mq.cuh"
+#include "select.cuh"
 #include "prefill.cuh"
 #include "prefill_swa.cuh"
 #include "prefill_ga.cuh"
@@ -558,6 +559,57 @@ mimo_status mimo_attn_cache_append(const mimo_shape* s, const void* k_chunk, con
   const long long items = static_cast<long long>(s->batch) * s->seqlen * s->n_kv_heads * 40;
   const long long blocks = std::min<long long>((items + 255) / 256, 4LL * sm_count_for(dev));
   mimo::cache_append_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(prm);
+  return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ERR_CUDA;
+}
+
+size_t mimo_attn_select_workspace_size(const mimo_shape* s, int cache_capacity) {
+  if (check_heads(s) != MIMO_OK || cache_capacity < 1) return 0;
+  const size_t n = static_cast<size_t>(s->batch) * s->n_kv_heads * cache_capacity * sizeof(uint32_t);
+  return (n + 255) / 256 * 256;
+}
+
+mimo_status mimo_attn_select_tokens(const mimo_shape* s, const void* q, const void* k_cache,
+                                    int cache_capacity, long long seq_stride_tokens,
+                                    const int* lengths, int recent, int n_sel, int* sel_idx,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
+  mimo_status e = check_heads(s);
+  if (e != MIMO_OK) return e;
+  if (!q || !k_cache || !lengths || (n_sel > 0 && !sel_idx)) return MIMO_ERR_NULL;
+  if (cache_capacity < 1 || seq_stride_tokens < cache_capacity || recent < 0 || n_sel < 0)
+    return MIMO_ERR_SHAPE;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(lengths, 4) || (sel_idx && !aligned(sel_idx, 4)))
+    return MIMO_ERR_ALIGN;
+  const size_t need = mimo_attn_select_workspace_size(s, cache_capacity);
+  if (!workspace || workspace_bytes < need) return MIMO_ERR_WORKSPACE;
+  if (!aligned(workspace, 16)) return MIMO_ERR_ALIGN;
+  if (n_sel == 0) return MIMO_OK;
+  if (s->n_kv_heads > 65535 || s->batch > 65535) return MIMO_ERR_UNSUPPORTED;
+  if (current_device() < 0) return MIMO_ERR_CUDA;
+  mimo::SelectParams prm{};
+  prm.q = static_cast<const __nv_bfloat16*>(q);
+  prm.k = static_cast<const __nv_bfloat16*>(k_cache);
+  prm.lengths = lengths;
+  prm.keys = static_cast<uint32_t*>(workspace);
+  prm.sel = sel_idx;
+  prm.seq_stride = seq_stride_tokens;
+  prm.B = s->batch;
+  prm.Hq = s->n_q_heads;
+  prm.Hkv = s->n_kv_heads;
+  prm.cap = cache_capacity;
+  prm.recent = recent;
+  prm.n_sel = n_sel;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int cand = std::max(1, cache_capacity - recent);
+  const dim3 grid((cand + mimo::kSelScoreThreads - 1) / mimo::kSelScoreThreads, s->n_kv_heads, s->batch);
+  switch (s->n_q_heads / s->n_kv_heads) {
+    case 1: mimo::select_score_kernel<1><<<grid, mimo::kSelScoreThreads, 0, st>>>(prm); break;
+    case 2: mimo::select_score_kernel<2><<<grid, mimo::kSelScoreThreads, 0, st>>>(prm); break;
+    case 4: mimo::select_score_kernel<4><<<grid, mimo::kSelScoreThreads, 0, st>>>(prm); break;
+    case 8: mimo::select_score_kernel<8><<<grid, mimo::kSelScoreThreads, 0, st>>>(prm); break;
+    default: mimo::select_score_kernel<16><<<grid, mimo::kSelScoreThreads, 0, st>>>(prm); break;
+  }
+  if (cudaGetLastError() != cudaSuccess) return MIMO_ERR_CUDA;
+  mimo::select_topk_kernel<<<dim3(s->n_kv_heads, s->batch), mimo::kSelThreads, 0, st>>>(prm);
   return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ERR_CUDA;
 }
 

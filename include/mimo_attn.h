@@ -263,6 +263,32 @@ mimo_status mimo_attn_sparse_fp8(const mimo_shape* shape, const void* q, const v
                                  void* out, float* lse, void* workspace, size_t workspace_bytes,
                                  void* stream);
 
+/*
+ * Token selection for mimo_attn_sparse ("小米MiMo-V3的核心架构HySparse2" §二.2 / §四.3: token
+ * level, reused from the preceding full-attention layer, no trained retrieval module; the
+ * pages give no scoring rule - this is the library's). For sequence b and KV head g, every
+ * token t in [0, L_b - recent) scores max over the group's query heads of q_h . k_t; the
+ * n_sel best are kept (equal scores: lower t first) and written in increasing t, which is
+ * the sel_idx layout mimo_attn_sparse reads.
+ *
+ *  q        [B, Hq, 192] bf16 device (rotated), e.g. the query of the preceding GA layer
+ *  k_cache  [B, seq_stride_tokens, Hkv, 192] bf16 device, linear cache of rotated K
+ *  lengths  [B] int32 device (clamped to cache_capacity)
+ *  sel_idx  [B, Hkv, n_sel] int32 device (written); rows with fewer than n_sel candidates
+ *           hold all of them followed by -1 (a precondition violation for mimo_attn_sparse)
+ *  workspace  at least mimo_attn_select_workspace_size(shape, cache_capacity) bytes
+ *
+ * Two launches: a score pass (one thread per candidate, fp32 dot products) and one CTA per
+ * (b, g) doing a radix select and an ordered compaction. Errors: MIMO_ERR_NULL,
+ * MIMO_ERR_SHAPE (capacity, stride, recent or n_sel out of range), MIMO_ERR_ALIGN,
+ * MIMO_ERR_WORKSPACE, MIMO_ERR_UNSUPPORTED (batch or Hkv above 65535), MIMO_ERR_CUDA.
+ */
+mimo_status mimo_attn_select_tokens(const mimo_shape* shape, const void* q, const void* k_cache,
+                                    int cache_capacity, long long seq_stride_tokens,
+                                    const int* lengths, int recent, int n_sel, int* sel_idx,
+                                    void* workspace, size_t workspace_bytes, void* stream);
+size_t mimo_attn_select_workspace_size(const mimo_shape* shape, int cache_capacity);
+
 /* Bytes of device workspace mimo_attn_decode / mimo_attn_sparse need for these sizes
  * on the current device (0 when none is needed). Returns 0 for invalid arguments. */
 size_t mimo_attn_workspace_size(const mimo_shape* shape, int op, int cache_kind,

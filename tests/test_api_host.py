@@ -177,3 +177,21 @@ def test_prefill_chunk_and_append_reject_before_launch(L):
     assert app(kc=None) == 1
     assert app(stride=999) == 2
     assert app(kc=P(0x10008)) == 4
+
+
+def test_select_tokens_rejects_before_launch(L):
+    s = _shape(hq=64, hkv=4)
+    sel = lambda **kw: L.mimo_attn_select_tokens(  # noqa: E731
+        ctypes.byref(s), kw.get("q", GOOD), GOOD, kw.get("cap", 4096), kw.get("stride", 4096), GOOD,
+        kw.get("recent", 128), kw.get("n_sel", 1024), kw.get("out", GOOD), kw.get("ws", GOOD),
+        kw.get("wsb", 1 << 30), None)
+    assert sel(q=None) == 1
+    assert sel(out=None) == 1
+    assert sel(recent=-1) == 2
+    assert sel(n_sel=-5) == 2
+    assert sel(stride=100) == 2
+    assert sel(ws=None) == 5
+    assert sel(wsb=16) == 5
+    assert sel(q=P(0x10002)) == 4
+    need = L.mimo_attn_select_workspace_size(ctypes.byref(s), 4096)
+    assert need == 1 * 4 * 4096 * 4
