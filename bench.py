@@ -525,6 +525,35 @@ def bench_fp8_decode_step(steps, warmup, peaks, tag, dev, stream):
     return res
 
 
+def bench_select(steps, warmup, peaks, tag, dev, stream):
+    """Token selection on the sparse-decode shape: B=8, L=262144, 64Q/4KV, recent 128, 1024
+    selected per (sequence, KV head). Algorithmic bytes: every candidate K row once (384 B),
+    the score keys written once and read by the select pass (4 x 4 B)."""
+    from hybrid_sliding_window_sink_b200 import _lib
+    c = wl.SPARSE_DECODE
+    lengths = [c.context] * c.batch
+    d = wl.decode_inputs(c.batch, c.hq, c.hkv, c.context, lengths, seed=c.seed + 3, device=dev)
+    del d["v_cache"]
+    out = torch.empty(c.batch, c.hkv, c.n_sel, dtype=torch.int32, device=dev)
+    shape = _lib.make_shape(c.batch, 1, c.hq, c.hkv)
+    ws = torch.empty(int(_lib.lib().mimo_attn_select_workspace_size(ctypes.byref(shape), c.context)),
+                     dtype=torch.uint8, device=dev)
+
+    def step():
+        _lib.select_tokens(d["q"], d["k_cache"], d["lengths"], recent=c.recent, n_sel=c.n_sel,
+                           out=out, workspace=ws, stream=stream)
+
+    ms = timed(step, steps, warmup, stream) / steps
+    cand = (c.context - c.recent) * c.batch * c.hkv
+    bytes_ = float(cand * (wl.DQK * 2 + 4 * 4))
+    res = {"value": round(bytes_ / (ms * 1e-3) / 1e9, 1), "unit": "GB/s", "ms_per_call": round(ms, 4),
+           "bytes_per_call": bytes_, "launches_per_call": 2,
+           "roofline": roofline_hbm(bytes_, ms, peaks, tag),
+           "workload": "token selection B=8 L=262144 64Q/4KV, top 1024 outside the recent 128"}
+    del d, ws, out
+    return res
+
+
 def bench_sparse(steps, warmup, peaks, tag, dev, stream, calls=16):
     """Token-level sparse decode: ``calls`` independent calls (distinct q and index sets,
     >= 385 MB of gathered rows in all, more than L2) per step, captured in a CUDA graph."""
@@ -711,6 +740,11 @@ def main():
             torch.cuda.empty_cache()
         except Exception as e:
             wls["mtp_decode_step"] = {"error": repr(e)}
+        try:
+            wls["token_select"] = bench_select(max(3, ksteps), 3, peaks, tag, dev, stream)
+            torch.cuda.empty_cache()
+        except Exception as e:
+            wls["token_select"] = {"error": repr(e)}
         try:
             wls["sparse_decode"] = bench_sparse(max(5, ksteps), 3, peaks, tag, dev, stream)
             wls["sparse_decode"]["workload"] = wl.SPARSE_DECODE.name

@@ -564,7 +564,11 @@ mimo_status mimo_attn_cache_append(const mimo_shape* s, const void* k_chunk, con
 
 size_t mimo_attn_select_workspace_size(const mimo_shape* s, int cache_capacity) {
   if (check_heads(s) != MIMO_OK || cache_capacity < 1) return 0;
-  const size_t n = static_cast<size_t>(s->batch) * s->n_kv_heads * cache_capacity * sizeof(uint32_t);
+  // score keys [B, Hkv, round_up(cap, 4)] u32, then top-byte histograms [B, Hkv, chunks, 256] u16
+  const size_t bg = static_cast<size_t>(s->batch) * s->n_kv_heads;
+  const size_t keys = bg * ((static_cast<size_t>(cache_capacity) + 3) / 4 * 4) * sizeof(uint32_t);
+  const size_t chunks = (static_cast<size_t>(cache_capacity) + mimo::kSelChunk - 1) / mimo::kSelChunk;
+  const size_t n = keys + bg * chunks * 256 * sizeof(uint16_t);
   return (n + 255) / 256 * 256;
 }
 
@@ -590,6 +594,10 @@ mimo_status mimo_attn_select_tokens(const mimo_shape* s, const void* q, const vo
   prm.k = static_cast<const __nv_bfloat16*>(k_cache);
   prm.lengths = lengths;
   prm.keys = static_cast<uint32_t*>(workspace);
+  prm.key_stride = (cache_capacity + 3) / 4 * 4;
+  prm.n_chunks = (cache_capacity + mimo::kSelChunk - 1) / mimo::kSelChunk;
+  prm.hist = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(workspace) +
+                                         static_cast<size_t>(s->batch) * s->n_kv_heads * prm.key_stride * 4);
   prm.sel = sel_idx;
   prm.seq_stride = seq_stride_tokens;
   prm.B = s->batch;
@@ -600,14 +608,25 @@ mimo_status mimo_attn_select_tokens(const mimo_shape* s, const void* q, const vo
   prm.n_sel = n_sel;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const int cand = std::max(1, cache_capacity - recent);
-  const dim3 grid((cand + mimo::kSelScoreThreads - 1) / mimo::kSelScoreThreads, s->n_kv_heads, s->batch);
+  const dim3 grid((cand + mimo::kSelChunk - 1) / mimo::kSelChunk, s->n_kv_heads, s->batch);
+  auto launch = [&](auto kern) -> bool {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, mimo::kSelScoreSmem) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return false;
+    }
+    kern<<<grid, mimo::kDecThreads, mimo::kSelScoreSmem, st>>>(prm);
+    return true;
+  };
+  bool launched;
   switch (s->n_q_heads / s->n_kv_heads) {
-    case 1: mimo::select_score_kernel<1><<<grid, mimo::kSelScoreThreads, 0, st>>>(prm); break;
-    case 2: mimo::select_score_kernel<2><<<grid, mimo::kSelScoreThreads, 0, st>>>(prm); break;
-    case 4: mimo::select_score_kernel<4><<<grid, mimo::kSelScoreThreads, 0, st>>>(prm); break;
-    case 8: mimo::select_score_kernel<8><<<grid, mimo::kSelScoreThreads, 0, st>>>(prm); break;
-    default: mimo::select_score_kernel<16><<<grid, mimo::kSelScoreThreads, 0, st>>>(prm); break;
+    case 1: launched = launch(mimo::select_score_kernel<1>); break;
+    case 2: launched = launch(mimo::select_score_kernel<2>); break;
+    case 4: launched = launch(mimo::select_score_kernel<4>); break;
+    case 8: launched = launch(mimo::select_score_kernel<8>); break;
+    default: launched = launch(mimo::select_score_kernel<16>); break;
   }
+  if (!launched) return MIMO_ERR_CUDA;
   if (cudaGetLastError() != cudaSuccess) return MIMO_ERR_CUDA;
   mimo::select_topk_kernel<<<dim3(s->n_kv_heads, s->batch), mimo::kSelThreads, 0, st>>>(prm);
   return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ERR_CUDA;

@@ -7,11 +7,12 @@
 // (the attention logit up to the positive softmax scale, which does not change the order);
 // the n_sel best are kept, equal scores in increasing t, and listed in increasing t.
 //
-// select_score_kernel: one thread per candidate token, the group's queries in shared memory
-// as fp32, the key row read with 16-byte loads; writes an order-preserving uint32 of the
-// fp32 score. select_topk_kernel: one CTA per (b, g); a 4-pass radix select (8 bits per
-// pass, most significant first) finds the n_sel-th largest key T and how many keys equal to
-// T are needed; an ordered compaction (block scans over 1024 candidates at a time) keeps
+// select_score_kernel: 1024 candidates per CTA, S = Q K^T on the tensor cores (mma.sync,
+// fp32 accumulation) and the max over the group's heads; writes an order-preserving uint32
+// of the fp32 score and a histogram of its top byte per CTA. select_topk_kernel: one CTA per
+// (b, g); a 4-digit radix select (8 bits per digit, most significant first; the first digit's
+// histogram comes from the score pass) finds the n_sel-th largest key T and how many keys
+// equal to T are needed; an ordered compaction (one block scan per 16384 candidates) keeps
 // every key > T and the first needed keys == T, writing their indices in increasing order.
 #pragma once
 
@@ -20,17 +21,24 @@
 
 namespace mimo {
 
-constexpr int kSelScoreThreads = 256;
+constexpr int kSelChunk = 1024;   // candidate keys per score CTA
+constexpr int kSelScoreSmem = 2 * kDecSub * kKRow + 256 * 4;   // two 64-key K subtiles + histogram
 constexpr int kSelThreads = 1024;
+constexpr int kSelPerThread = 16;                 // candidates per thread per compaction step
+constexpr int kSelBlockKeys = kSelPerThread * kSelThreads;
+constexpr int kSelUnroll = 8;                     // 16-byte key loads in flight per thread
 
 struct SelectParams {
   const __nv_bfloat16* q;     // [B, Hq, 192]
   const __nv_bfloat16* k;     // [B, seq_stride, Hkv, 192]
   const int* lengths;         // [B]
-  uint32_t* keys;             // workspace [B, Hkv, cap]: order-preserving score bits
+  uint32_t* keys;             // workspace [B, Hkv, key_stride]: order-preserving score bits
+  uint16_t* hist;             // workspace [B, Hkv, n_chunks, 256]: top-byte histogram per score CTA
   int* sel;                   // [B, Hkv, n_sel]
   long long seq_stride;
   int B, Hq, Hkv, cap, recent, n_sel;
+  int key_stride;             // cap rounded up to a multiple of 4 (16-byte aligned rows)
+  int n_chunks;               // ceil(cap / kSelChunk)
 };
 
 __device__ __forceinline__ int sel_candidates(const SelectParams& p, int b) {
@@ -46,36 +54,108 @@ __device__ __forceinline__ uint32_t order_key(float x) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// Scores of 1024 candidate keys per CTA as a small GEMM on the tensor cores: K rows are
+// gathered by 16-byte cp.async into double-buffered 64-key subtiles (rows XOR-swizzled for
+// ldmatrix, as in the decode kernel), each warp takes 16 keys per subtile and computes
+// S = Q K^T with m16n8k16 bf16 MMAs (the group's <= 16 heads as M, zero rows masked), then
+// the max over the heads per key.
 template <int G>
-__global__ void __launch_bounds__(kSelScoreThreads) select_score_kernel(const SelectParams p) {
-  __shared__ float s_q[G * kDQK];
+__global__ void __launch_bounds__(kDecThreads, 4) select_score_kernel(const SelectParams p) {
+  extern __shared__ __align__(1024) uint8_t smem[];
   const int g = blockIdx.y, b = blockIdx.z;
-  const __nv_bfloat16* qg = p.q + (static_cast<long long>(b) * p.Hq + g * G) * kDQK;
-  for (int i = threadIdx.x; i < G * kDQK; i += kSelScoreThreads) s_q[i] = __bfloat162float(qg[i]);
-  __syncthreads();
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int gq = lane >> 2, tq = lane & 3;
   const int hi = sel_candidates(p, b);
-  const int t = blockIdx.x * kSelScoreThreads + threadIdx.x;
-  if (t >= hi) return;
-  const __nv_bfloat16* krow = p.k + ((static_cast<long long>(b) * p.seq_stride + t) * p.Hkv + g) * kDQK;
-  float acc[G];
+  const int k_begin = blockIdx.x * kSelChunk;
+  if (k_begin >= hi) return;
+  const int n_here = min(kSelChunk, hi - k_begin);
+  const uint32_t s_base = smem_u32(smem);
+  int* s_h = reinterpret_cast<int*>(smem + 2 * kDecSub * kKRow);
+  for (int i = tid; i < 256; i += kDecThreads) s_h[i] = 0;   // first use is after a barrier
+  const __nv_bfloat16* kbase = p.k + (static_cast<long long>(b) * p.seq_stride) * p.Hkv * kDQK + g * kDQK;
+  const long long krow_stride = static_cast<long long>(p.Hkv) * kDQK;
+  auto load_sub = [&](int st, int stage) {
+    const uint32_t sK = s_base + stage * (kDecSub * kKRow);
 #pragma unroll
-  for (int h = 0; h < G; ++h) acc[h] = 0.f;
-#pragma unroll 4
-  for (int u = 0; u < kDQK / 8; ++u) {
-    const uint4 x = __ldg(reinterpret_cast<const uint4*>(krow) + u);
-    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+    for (int i = 0; i < (kDecSub * 24) / kDecThreads; ++i) {
+      const int idx = tid + i * kDecThreads;
+      const int row = idx / 24, u = idx - row * 24;
+      const int key = st * kDecSub + row;
+      const bool ok = key < n_here;
+      const int t = ok ? k_begin + key : 0;
+      cp_async16(sK + row * kKRow + ((u ^ (row & 7)) << 4), kbase + t * krow_stride + u * 8, ok ? 16u : 0u);
+    }
+  };
+  const int nsub = (n_here + kDecSub - 1) / kDecSub;
+  load_sub(0, 0);
+  cp_async_commit();
+  if (nsub > 1) load_sub(1, 1);
+  cp_async_commit();
+  uint32_t qa[12][4];
+  {
+    const __nv_bfloat16* qg = p.q + (static_cast<long long>(b) * p.Hq + g * G) * kDQK;
+    const bool r0ok = gq < G, r1ok = gq + 8 < G;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float k0 = bf16_lo(w[e]), k1 = bf16_hi(w[e]);
-      const int d = u * 8 + 2 * e;
-#pragma unroll
-      for (int h = 0; h < G; ++h) acc[h] = fmaf(s_q[h * kDQK + d + 1], k1, fmaf(s_q[h * kDQK + d], k0, acc[h]));
+    for (int kk = 0; kk < 12; ++kk) {
+      const int d0 = kk * 16 + tq * 2;
+      qa[kk][0] = r0ok ? *reinterpret_cast<const uint32_t*>(qg + gq * kDQK + d0) : 0u;
+      qa[kk][1] = r1ok ? *reinterpret_cast<const uint32_t*>(qg + (gq + 8) * kDQK + d0) : 0u;
+      qa[kk][2] = r0ok ? *reinterpret_cast<const uint32_t*>(qg + gq * kDQK + d0 + 8) : 0u;
+      qa[kk][3] = r1ok ? *reinterpret_cast<const uint32_t*>(qg + (gq + 8) * kDQK + d0 + 8) : 0u;
     }
   }
-  float best = acc[0];
+  uint32_t* keys = p.keys + (static_cast<long long>(b) * p.Hkv + g) * p.key_stride + k_begin;
+  const int mi = lane >> 3, r8 = lane & 7;
+  for (int st = 0; st < nsub; ++st) {
+    cp_async_wait<1>();
+    __syncthreads();
+    const uint32_t sK = s_base + (st & 1) * (kDecSub * kKRow);
+    float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    const int krow = warp * 16 + ((mi >> 1) << 3) + r8;
+    const uint32_t rowaddr = sK + krow * kKRow;
 #pragma unroll
-  for (int h = 1; h < G; ++h) best = fmaxf(best, acc[h]);
-  p.keys[(static_cast<long long>(b) * p.Hkv + g) * p.cap + t] = order_key(best);
+    for (int kk = 0; kk < 12; ++kk) {
+      const int unit = 2 * kk + (mi & 1);
+      uint32_t b00, b01, b10, b11;
+      ldmatrix_x4(rowaddr + ((unit ^ (krow & 7)) << 4), b00, b01, b10, b11);
+      mma_16816(sacc[0], qa[kk], b00, b01);
+      mma_16816(sacc[1], qa[kk], b10, b11);
+    }
+    // sacc[nt][e]: head row gq (e < 2) or gq + 8 (e >= 2), key nt*8 + 2 tq + (e & 1)
+    float mx[2][2];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const float a = gq < G ? sacc[nt][c] : -INFINITY;
+        const float bb = gq + 8 < G ? sacc[nt][c + 2] : -INFINITY;
+        float m = fmaxf(a, bb);
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));    // over gq
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 8));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 16));
+        mx[nt][c] = m;
+      }
+    if (gq == 0) {
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int key = st * kDecSub + warp * 16 + nt * 8 + 2 * tq + c;
+          if (key < n_here) {
+            const uint32_t u = order_key(mx[nt][c]);
+            keys[key] = u;
+            atomicAdd(&s_h[u >> 24], 1);
+          }
+        }
+    }
+    __syncthreads();
+    if (st + 2 < nsub) load_sub(st + 2, st & 1);
+    cp_async_commit();
+  }
+  cp_async_wait<0>();
+  // first radix digit of this chunk's keys, read back by select_topk_kernel (counts <= 1024)
+  uint16_t* h = p.hist + ((static_cast<long long>(b) * p.Hkv + g) * p.n_chunks + blockIdx.x) * 256;
+  for (int i = tid; i < 256; i += kDecThreads) h[i] = static_cast<uint16_t>(s_h[i]);
 }
 
 // Block-wide exclusive scan of one int per thread (1024 threads); returns the block total.
@@ -107,63 +187,158 @@ __device__ __forceinline__ int block_exclusive_scan(int x, int& total, int* s_wa
   return res;
 }
 
+// Picks the radix bin holding the need-th largest key among the 256 bins of s_hist (warp 0):
+// lane l owns bins 255-8l .. 248-8l, a shuffle scan counts the keys in higher lanes' bins.
+__device__ __forceinline__ void select_pick_bin(const int* s_hist, int shift, uint32_t prefix, int need,
+                                                uint32_t* s_prefix, int* s_need) {
+  const int lane = threadIdx.x & 31;
+  int c[8];
+  int tot = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    c[j] = s_hist[255 - 8 * lane - j];
+    tot += c[j];
+  }
+  int incl = tot;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const int excl = incl - tot;
+  const unsigned own = __ballot_sync(0xffffffffu, excl < need && need <= incl);
+  const int owner = own ? __ffs(own) - 1 : 31;   // the counts always place need in one lane
+  if (lane == owner) {
+    int above = excl, j = 0;
+    for (; j < 7; ++j) {
+      if (above + c[j] >= need) break;
+      above += c[j];
+    }
+    *s_prefix = prefix | (static_cast<uint32_t>(255 - 8 * lane - j) << shift);
+    *s_need = need - above;
+  }
+}
+
 __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const SelectParams p) {
   __shared__ int s_hist[256];
   __shared__ int s_warp[33];
   __shared__ uint32_t s_prefix;
   __shared__ int s_need;
   const int g = blockIdx.x, b = blockIdx.y;
+  const int tid = threadIdx.x;
   const int hi = sel_candidates(p, b);
-  const uint32_t* keys = p.keys + (static_cast<long long>(b) * p.Hkv + g) * p.cap;
-  int* out = p.sel + (static_cast<long long>(b) * p.Hkv + g) * p.n_sel;
+  const long long bg = static_cast<long long>(b) * p.Hkv + g;
+  const uint32_t* keys = p.keys + bg * p.key_stride;
+  const uint4* keys4 = reinterpret_cast<const uint4*>(keys);
+  int* out = p.sel + bg * p.n_sel;
   const int k = p.n_sel < hi ? p.n_sel : hi;   // fewer candidates than n_sel: keep them all
+  const int n4 = (hi + 3) >> 2;
 
   // radix select: T = the k-th largest key; need = how many keys equal to T are kept
   uint32_t prefix = 0, mask = 0;
   int need = k;
   if (k > 0 && k < hi) {
-    for (int shift = 24; shift >= 0; shift -= 8) {
-      for (int i = threadIdx.x; i < 256; i += kSelThreads) s_hist[i] = 0;
-      __syncthreads();
-      for (int i = threadIdx.x; i < hi; i += kSelThreads) {
-        const uint32_t u = keys[i];
-        if ((u & mask) == prefix) atomicAdd(&s_hist[(u >> shift) & 0xFFu], 1);
-      }
-      __syncthreads();
-      if (threadIdx.x == 0) {
-        int above = 0, bin = 255;
-        for (; bin > 0; --bin) {
-          if (above + s_hist[bin] >= need) break;
-          above += s_hist[bin];
+    {  // digit 1 (bits 31..24): sum the score kernel's per-chunk histograms; lane l of warp w
+       // adds bins 8l..8l+7 (one 16-byte load) of chunks w, w + 32, ...
+      const int nch = (hi + kSelChunk - 1) / kSelChunk;
+      const uint4* h4 = reinterpret_cast<const uint4*>(p.hist + bg * p.n_chunks * 256);
+      const int lane = tid & 31, warp = tid >> 5;
+      if (tid < 256) s_hist[tid] = 0;
+      int acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll 4
+      for (int c = warp; c < nch; c += kSelThreads / 32) {
+        const uint4 v = h4[c * 32 + lane];
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          acc[2 * e] += static_cast<int>(w[e] & 0xFFFFu);
+          acc[2 * e + 1] += static_cast<int>(w[e] >> 16);
         }
-        s_prefix = prefix | (static_cast<uint32_t>(bin) << shift);
-        s_need = need - above;
       }
+      __syncthreads();
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        if (acc[e]) atomicAdd(&s_hist[8 * lane + e], acc[e]);
+      __syncthreads();
+      if (tid < 32) select_pick_bin(s_hist, 24, prefix, need, &s_prefix, &s_need);
+      __syncthreads();
+      prefix = s_prefix;
+      need = s_need;
+      mask = 0xFF000000u;
+    }
+    for (int shift = 16; shift >= 0; shift -= 8) {
+      if (tid < 256) s_hist[tid] = 0;
+      __syncthreads();
+      for (int i4 = tid; i4 < n4; i4 += kSelUnroll * kSelThreads) {
+        uint4 v[kSelUnroll];
+#pragma unroll
+        for (int r = 0; r < kSelUnroll; ++r) {
+          const int j = i4 + r * kSelThreads;
+          v[r] = j < n4 ? keys4[j] : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int r = 0; r < kSelUnroll; ++r) {
+          const int i0 = 4 * (i4 + r * kSelThreads);
+          const uint32_t u[4] = {v[r].x, v[r].y, v[r].z, v[r].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (i0 + e < hi && (u[e] & mask) == prefix) atomicAdd(&s_hist[(u[e] >> shift) & 0xFFu], 1);
+        }
+      }
+      __syncthreads();
+      if (tid < 32) select_pick_bin(s_hist, shift, prefix, need, &s_prefix, &s_need);
       __syncthreads();
       prefix = s_prefix;
       need = s_need;
       mask |= 0xFFu << shift;
-      __syncthreads();
     }
   }
   const bool take_all = k >= hi;
-  // ordered compaction over the candidates in increasing index
+  // ordered compaction, 16 consecutive candidates per thread: one block scan per step of the
+  // packed counts (keys == T in the high half, keys > T in the low half; each <= 16384)
   int out_base = 0, tie_base = 0;
-  for (int base = 0; base < hi; base += kSelThreads) {
-    const int i = base + threadIdx.x;
-    const uint32_t u = i < hi ? keys[i] : 0u;
-    const bool valid = i < hi;
-    const int eq = valid && !take_all && u == prefix ? 1 : 0;
-    int eq_total;
-    const int eq_rank = block_exclusive_scan(eq, eq_total, s_warp);
-    const int take = valid && (take_all || u > prefix || (eq && tie_base + eq_rank < need)) ? 1 : 0;
-    int take_total;
-    const int pos = block_exclusive_scan(take, take_total, s_warp);
-    if (take && out_base + pos < p.n_sel) out[out_base + pos] = i;
-    out_base += take_total;
+  for (int base = 0; base < hi; base += kSelBlockKeys) {
+    const int i0 = base + kSelPerThread * tid;
+    uint4 v[kSelPerThread / 4];
+#pragma unroll
+    for (int r = 0; r < kSelPerThread / 4; ++r)
+      v[r] = i0 + 4 * r < hi ? keys4[(i0 >> 2) + r] : make_uint4(0u, 0u, 0u, 0u);
+    uint32_t gt = 0, eq = 0;   // bit e: candidate i0 + e
+#pragma unroll
+    for (int r = 0; r < kSelPerThread / 4; ++r) {
+      const uint32_t u[4] = {v[r].x, v[r].y, v[r].z, v[r].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int idx = i0 + 4 * r + e;
+        const bool valid = idx < hi;
+        if (valid && (take_all || u[e] > prefix)) gt |= 1u << (4 * r + e);
+        if (valid && !take_all && u[e] == prefix) eq |= 1u << (4 * r + e);
+      }
+    }
+    const int ngt = __popc(gt), neq = __popc(eq);
+    int total;
+    const int excl = block_exclusive_scan((neq << 16) | ngt, total, s_warp);
+    const int rem = need - tie_base > 0 ? need - tie_base : 0;   // ties still to keep
+    if (gt | eq) {
+      int e_seen = excl >> 16;
+      int pos = out_base + (excl & 0xFFFF) + (e_seen < rem ? e_seen : rem);
+      uint32_t m = gt | eq;
+      while (m) {
+        const int e = __ffs(m) - 1;
+        m &= m - 1;
+        bool take = true;
+        if ((eq >> e) & 1u) take = e_seen++ < rem;
+        if (take) {
+          if (pos < p.n_sel) out[pos] = i0 + e;
+          ++pos;
+        }
+      }
+    }
+    const int eq_total = total >> 16;
+    out_base += (total & 0xFFFF) + (eq_total < rem ? eq_total : rem);
     tie_base += eq_total;
   }
-  for (int j = out_base + threadIdx.x; j < p.n_sel; j += kSelThreads) out[j] = -1;   // too few candidates
+  for (int j = out_base + tid; j < p.n_sel; j += kSelThreads) out[j] = -1;   // too few candidates
 }
 
 }  // namespace mimo

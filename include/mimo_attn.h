@@ -278,8 +278,11 @@ mimo_status mimo_attn_sparse_fp8(const mimo_shape* shape, const void* q, const v
  *           hold all of them followed by -1 (a precondition violation for mimo_attn_sparse)
  *  workspace  at least mimo_attn_select_workspace_size(shape, cache_capacity) bytes
  *
- * Two launches: a score pass (one thread per candidate, fp32 dot products) and one CTA per
- * (b, g) doing a radix select and an ordered compaction. Errors: MIMO_ERR_NULL,
+ * Two launches: a score pass (1,024 candidates per CTA; q . k on the tensor cores with fp32
+ * accumulation, writing an order-preserving key per candidate and a histogram of its top
+ * byte) and one CTA per (b, g) doing a radix select and an ordered compaction. The
+ * workspace holds the keys, [B, Hkv, cache_capacity rounded up to 4] uint32, followed by
+ * the histograms, [B, Hkv, ceil(cache_capacity / 1024), 256] uint16. Errors: MIMO_ERR_NULL,
  * MIMO_ERR_SHAPE (capacity, stride, recent or n_sel out of range), MIMO_ERR_ALIGN,
  * MIMO_ERR_WORKSPACE, MIMO_ERR_UNSUPPORTED (batch or Hkv above 65535), MIMO_ERR_CUDA.
  */

@@ -194,4 +194,6 @@ def test_select_tokens_rejects_before_launch(L):
     assert sel(wsb=16) == 5
     assert sel(q=P(0x10002)) == 4
     need = L.mimo_attn_select_workspace_size(ctypes.byref(s), 4096)
-    assert need == 1 * 4 * 4096 * 4
+    assert need == 1 * 4 * 4096 * 4 + 1 * 4 * 4 * 256 * 2      # keys, then top-byte histograms
+    # key rows padded to 16 bytes
+    assert L.mimo_attn_select_workspace_size(ctypes.byref(s), 1027) == (4 * 1028 * 4 + 4 * 2 * 512 + 255) // 256 * 256
