@@ -273,7 +273,7 @@ def bench_chunk_prefill(steps, warmup, peaks, tag, dev, stream, chunk=16384, pre
         del inp, q, out, lse
         torch.cuda.empty_cache()
     res["workload"] = f"chunked prefill, {chunk}-token chunk after a {prefix}-token prefix (rotated), B=1"
-    res["kernel"] = "generic tcgen05 prefill kernel (one compute warpgroup)"
+    res["kernel"] = {"swa": "prefill_swa_kernel (K/V ring)", "ga": "prefill_ga_kernel (row-block pairs)"}
     return res
 
 

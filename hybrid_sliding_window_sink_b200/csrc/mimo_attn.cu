@@ -157,9 +157,11 @@ mimo_status launch_prefill_swa(const mimo_shape* s, const void* q, const void* k
   using L = mimo::SwaLayout;
   CUtensorMap tq, tk, tv;
   const uint64_t n = static_cast<uint64_t>(s->seqlen), B = static_cast<uint64_t>(s->batch);
+  const uint64_t nk = static_cast<uint64_t>(prm.nk);   // keys: n, or prefix + chunk
+  if (prm.q_off % mimo::kSwaP != 0) return MIMO_ERR_UNSUPPORTED;
   if (!make_tmap(&tq, q, mimo::kDQK, s->n_q_heads, n, B, mimo::kSwaG, mimo::kSwaP) ||
-      !make_tmap(&tk, k, mimo::kDQK, s->n_kv_heads, n, B, 1, 16) ||
-      !make_tmap(&tv, v, mimo::kDV, s->n_kv_heads, n, B, 1, 16))
+      !make_tmap(&tk, k, mimo::kDQK, s->n_kv_heads, nk, B, 1, 16) ||
+      !make_tmap(&tv, v, mimo::kDV, s->n_kv_heads, nk, B, 1, 16))
     return MIMO_ERR_CUDA;
   if (cudaFuncSetAttribute(mimo::prefill_swa_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            L::SMEM) != cudaSuccess) {
@@ -217,13 +219,16 @@ mimo_status prefill_group(const mimo_shape* s, const void* q, const void* k, con
   return launch_prefill<G, 128, 2>(s, q, k, v, prm, sms, st);
 }
 
-// Chunked prefill: GA layers with 8 or 16 query heads per KV head on the pair kernel, every
-// other shape on the generic kernel (query positions offset, keys from a prefix + the chunk).
+// Chunked prefill: GA layers with 8 or 16 query heads per KV head on the pair kernel, SWA
+// layers with 8 (W <= 129, chunk offset a multiple of 16) on the ring kernel, every other
+// shape on the generic kernel (query positions offset, keys from a prefix + the chunk).
 template <int G>
 mimo_status prefill_chunk_group(const mimo_shape* s, const void* q, const void* k, const void* v,
                                 const PrefillParams& prm, int sms, cudaStream_t st) {
   constexpr int P = 128 / G;
   const bool swa = prm.window > 0 && prm.window < prm.nk;
+  if (G == mimo::kSwaG && swa && prm.window <= 129 && prm.rot_dims <= 64 && prm.q_off % mimo::kSwaP == 0)
+    return launch_prefill_swa(s, q, k, v, prm, sms, st);
   if constexpr (G == 8 || G == 16) {   // full causal prefix: the pair kernel
     if (!swa && prm.rot_dims <= 64) return launch_prefill_ga<G>(s, q, k, v, prm, sms, st);
   }

@@ -7,6 +7,10 @@
 // lie in the 144-key span [p0 - 128, p0 + 16) (9 units of 16 keys), so one S tile
 // covers all of them and the softmax of a row block needs no rescaling across tiles.
 //
+// Chunked prefill: query row i of the call sits at position q_off + i (q_off a multiple of
+// 16, so blocks stay on 16-key units); keys come from a prefix + the chunk (nk rows), and
+// prefix rows below krot_from are stored rotated (their rotated dims only turn into f16).
+//
 // Layout of the work. Each persistent CTA takes a contiguous run of row blocks of the
 // flattened (sequence, KV head, block) order, so consecutive blocks share 128 of their
 // 144 keys. K and V live in a shared-memory ring of 11 units of 16 rows (176 rows):
@@ -221,8 +225,9 @@ __global__ void __launch_bounds__(kSwaThreads, 1)
       for (long long f = f0; f < f1 && ok; ++f) {
         const int bg = static_cast<int>(f / nqt), t = static_cast<int>(f % nqt);
         const int b = bg / p.Hkv, g = bg - b * p.Hkv;
+        const int ua = t + (p.q_off >> 4);   // K/V unit holding the block's own positions
         if (f == f0 || t == 0)
-          for (int u = t - 8; u < t && ok; ++u) ok = load_unit(b, g, u);
+          for (int u = ua - 8; u < ua && ok; ++u) ok = load_unit(b, g, u);
         if (!ok) break;
         const int st = nq & 1;
         if (nq >= 2 && !mbar_wait(bar(kSwQEmpty + st), ((nq >> 1) - 1) & 1, s_abort, err)) { ok = false; break; }
@@ -232,7 +237,7 @@ __global__ void __launch_bounds__(kSwaThreads, 1)
                       g * kSwaG, t * kSwaP, b);
         SWA_TRACE(nq, 9);
         ++nq;
-        ok = load_unit(b, g, t);
+        ok = load_unit(b, g, ua);
       }
       if (!ok) {   // let every issued copy land before the CTA can exit
         for (int s = seq - kSwaUnits < 0 ? 0 : seq - kSwaUnits; s < seq; ++s)
@@ -346,7 +351,7 @@ __global__ void __launch_bounds__(kSwaThreads, 1)
       const bool first = (f == f0 || t == 0);
       if (first) seq += 8;
       const int useq = seq++;
-      const int p0 = t * kSwaP;
+      const int p0 = p.q_off + t * kSwaP;            // absolute position of the block
       float2* tab = reinterpret_cast<float2*>(smem + L::OFF_TAB + (i & 1) * L::TAB_BYTES);
       if (ctid == 0) SWA_TRACE(i, 0);
       // (cos, sin) of the block's 16 positions (double buffered: tile i - 1 may still read)
@@ -364,7 +369,7 @@ __global__ void __launch_bounds__(kSwaThreads, 1)
       }
       if (!wait_all(bar(kSwQFull + (i & 1)), (i >> 1) & 1)) break;
       if (ctid == 0) SWA_TRACE(i, 1);
-      if (half > 0 && p0 + (ctid >> 3) < p.n)
+      if (half > 0 && t * kSwaP + (ctid >> 3) < p.n)
         rope_row_tab(smem + L::OFF_Q + (i & 1) * L::Q_STAGE + ctid * 128, ctid, nun,
                      tab + (ctid >> 3) * 32);
       // K units of this block: the new one, or the whole window at the start of a run
@@ -389,11 +394,12 @@ __global__ void __launch_bounds__(kSwaThreads, 1)
           for (int rr = ctid; rr < 16 * kSwaWin; rr += 128) {
             const int kpos = p0 - 128 + rr;
             const int ring_row = ((s_first + rr / 16) % kSwaUnits) * 16 + (rr & 15);
-            if (kpos >= 0 && kpos < p.n) rope_row(sK, L::R_CHUNK, ring_row, kpos, p.rot_dims, s_invf);
+            if (kpos >= p.krot_from && kpos < p.nk) rope_row(sK, L::R_CHUNK, ring_row, kpos, p.rot_dims, s_invf);
+            else if (kpos >= 0 && kpos < p.krot_from) f16_row(sK, L::R_CHUNK, ring_row, p.rot_dims);
           }
         } else if (ctid < 16) {
           const int ring_row = (useq % kSwaUnits) * 16 + ctid;
-          if (p0 + ctid < p.n)
+          if (p0 + ctid < p.nk)   // a block's own keys lie in the chunk: never stored rotated
             rope_row_tab(smem + L::OFF_K + ring_row * 128, ring_row, nun, tab + ctid * 32);
         }
       }
@@ -422,10 +428,11 @@ __global__ void __launch_bounds__(kSwaThreads, 1)
       const int useq = seq++;
       if ((i & 1) != w) continue;
       const int b = bg / p.Hkv, g = bg - b * p.Hkv;
-      const int p0 = t * kSwaP;
-      const int pos = p0 + pl;
+      const int qi = t * kSwaP + pl;                 // query row within the call
+      const int p0 = p.q_off + t * kSwaP;            // absolute positions
+      const int pos = p.q_off + qi;
       const int hq = g * kSwaG + hl;
-      const bool row_ok = pos < p.n;
+      const bool row_ok = qi < p.n;
 
       // Softmax over the row block's keys, two passes over TMEM. Slot block c (columns
       // 16c..16c+15) holds the unit d = (useq - c) mod 11 blocks back: keys kb + e with
@@ -538,7 +545,7 @@ __global__ void __launch_bounds__(kSwaThreads, 1)
       tc_fence_after();
       if (ctid == 0) SWA_TRACE(i, 5);
       const float inv_l = lt > 0.f ? sc / lt : 0.f;
-      __nv_bfloat16* orow = p.out + ((static_cast<long long>(b) * p.n + pos) * p.Hq + hq) * 128;
+      __nv_bfloat16* orow = p.out + ((static_cast<long long>(b) * p.n + qi) * p.Hq + hq) * 128;
       // O columns [128, 192) overlap the S columns of this group's next tile: read them
       // first, release the TMEM region, then finish with columns [192, 256)
 #pragma unroll 1
@@ -565,7 +572,7 @@ __global__ void __launch_bounds__(kSwaThreads, 1)
         }
       }
       if (row_ok && p.lse)
-        p.lse[(static_cast<long long>(b) * p.Hq + hq) * p.n + pos] =
+        p.lse[(static_cast<long long>(b) * p.Hq + hq) * p.n + qi] =
             lt > 0.f ? (M + log2f(lt)) * kLn2 : -INFINITY;
       if (ctid == 0) SWA_TRACE(i, 6);
     }

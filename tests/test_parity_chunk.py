@@ -29,6 +29,11 @@ def _rotated_prefix(k, off, theta, rot):
     (1, 200, 0, 64, 4, 0, True),           # no prefix: plain prefill
     (1, 64, 4097, 16, 1, 7, True),         # tiny window far into the sequence
     (1, 100, 150, 32, 8, 300, False),      # window longer than the chunk, shorter than the keys
+    # SWA ring kernel (8 heads per KV head, W <= 129, offset a multiple of 16)
+    (1, 300, 1024, 64, 8, 128, True),      # SWA layer layout, stored-rotated prefix
+    (2, 130, 16, 16, 2, 128, False),       # one raw prefix unit
+    (1, 97, 4096, 16, 2, 129, True),       # W = 129, ragged last block
+    (2, 1536, 2048, 64, 8, 128, True),     # long runs per CTA: ring units reused across blocks
 ])
 def test_prefill_chunk(cuda_device, B, n, off, hq, hkv, window, rotated):
     theta = wl.SWA_THETA if window > 0 else wl.GA_THETA
@@ -46,10 +51,11 @@ def test_prefill_chunk(cuda_device, B, n, off, hq, hkv, window, rotated):
     compare(wl.to_f64(out), o_ref, wl.to_f64(lse), l_ref, f"chunk off={off} n={n} W={window}")
 
 
-def test_chunks_match_whole_prefill(cuda_device):
+@pytest.mark.parametrize("cuts", [(0, 250, 511, 700), (0, 256, 512, 700)])
+def test_chunks_match_whole_prefill(cuda_device, cuts):
     """Three chunks (each reading the raw prefix) and one whole-sequence call both match the
-    oracle's whole-sequence rows (different kernels: the chunks run on the generic kernel,
-    the whole call on the SWA ring kernel)."""
+    oracle's whole-sequence rows (chunks at offsets that are multiples of 16 run on the SWA
+    ring kernel like the whole call, the others on the generic kernel)."""
     n, hq, hkv = 700, 16, 2
     inp = wl.prefill_inputs(1, n, hq, hkv, seed=1400)
     d = {k: v.to(cuda_device) for k, v in inp.items()}
@@ -58,7 +64,7 @@ def test_chunks_match_whole_prefill(cuda_device):
     whole, lw = _lib.prefill(d["q"], d["k"], d["v"], d["sink"], window=128, rope_theta=1e4, rot_dims=64)
     torch.cuda.synchronize()
     compare(wl.to_f64(whole), o_ref, wl.to_f64(lw), l_ref, "whole")
-    for a, b in ((0, 250), (250, 511), (511, 700)):
+    for a, b in zip(cuts[:-1], cuts[1:]):
         o, l = _lib.prefill_chunk(d["q"][:, a:b].contiguous(), d["k"][:, :b].contiguous(),
                                   d["v"][:, :b].contiguous(), d["sink"], pos_offset=a,
                                   k_prefix_rotated=False, window=128, rope_theta=1e4, rot_dims=64)
