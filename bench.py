@@ -548,7 +548,7 @@ def bench_select(steps, warmup, peaks, tag, dev, stream):
     bytes_ = float(cand * (wl.DQK * 2 + 4 * 4))
     res = {"value": round(bytes_ / (ms * 1e-3) / 1e9, 1), "unit": "GB/s", "ms_per_call": round(ms, 4),
            "bytes_per_call": bytes_, "launches_per_call": 2,
-           "roofline": roofline_hbm(bytes_, ms, peaks, tag),
+           "roofline": roofline_hbm(bytes_, ms, peaks, tag, traffic_for("token_select", cand)),
            "workload": "token selection B=8 L=262144 64Q/4KV, top 1024 outside the recent 128"}
     del d, ws, out
     return res

@@ -16,7 +16,11 @@ Cases:
   fp8_linear_b64_l16k   GA decode over an FP8 (E4M3 + per-row scale) linear cache, B=64, 16384
                         tokens (all full), 64 Q / 4 KV heads
   chunk_ga_c8192_p8192  GA chunked prefill: 8192-token chunk after an 8192-token rotated prefix,
-                        64 Q / 4 KV heads (generic prefill kernel)
+                        64 Q / 4 KV heads (row-block pair kernel)
+  chunk_swa_c8192_p8192 SWA chunked prefill: 8192-token chunk after an 8192-token rotated prefix,
+                        64 Q / 8 KV heads, W=128 (K/V-ring kernel)
+  select_b8_l65536      token selection, B=8, L=65536, 64 Q / 4 KV heads, the 1024 best
+                        outside the recent 128
 Prints the mean time per call over --reps calls (after two warm-up calls).
 """
 
@@ -80,6 +84,21 @@ def _case(name, dev):
         q = inp["q"][:, 8192:].contiguous()
         return lambda: _lib.prefill_chunk(q, inp["k"], inp["v"], inp["sink"], pos_offset=8192,
                                           k_prefix_rotated=True, window=0, rope_theta=1e7, rot_dims=64)
+    if name == "chunk_swa_c8192_p8192":
+        inp = wl.prefill_inputs(1, 16384, 64, 8, seed=13, device=dev)
+        q = inp["q"][:, 8192:].contiguous()
+        return lambda: _lib.prefill_chunk(q, inp["k"], inp["v"], inp["sink"], pos_offset=8192,
+                                          k_prefix_rotated=True, window=128, rope_theta=1e4, rot_dims=64)
+    if name == "select_b8_l65536":
+        L = 65536
+        d = wl.decode_inputs(8, 64, 4, L, [L] * 8, seed=14, device=dev)
+        del d["v_cache"]
+        out = torch.empty(8, 4, 1024, dtype=torch.int32, device=dev)
+        shape = _lib.make_shape(8, 1, 64, 4)
+        ws = torch.empty(int(_lib.lib().mimo_attn_select_workspace_size(ctypes.byref(shape), L)),
+                         dtype=torch.uint8, device=dev)
+        return lambda: _lib.select_tokens(d["q"], d["k_cache"], d["lengths"], recent=128, n_sel=1024,
+                                          out=out, workspace=ws)
     raise SystemExit(f"unknown case {name}")
 
 
