@@ -139,6 +139,25 @@ __device__ __forceinline__ void rope_half(uint8_t* row_base, int row, int nun, c
   }
 }
 
+// Rotates one 8-dim unit u (< nun) of the first half of a tile row and its partner u + nun.
+__device__ __forceinline__ void rope_unit(uint8_t* row_base, int row, int nun, const float4* t4, int u) {
+  uint4* px = reinterpret_cast<uint4*>(row_base + ((u ^ (row & 7)) << 4));
+  uint4* py = reinterpret_cast<uint4*>(row_base + (((u + nun) ^ (row & 7)) << 4));
+  const uint4 x = *px, y = *py;
+  uint32_t xs[4] = {x.x, x.y, x.z, x.w};
+  uint32_t ys[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+  for (int e2 = 0; e2 < 4; ++e2) {
+    const float4 cs = t4[u * 4 + e2];
+    const float x0 = bf16_lo(xs[e2]), x1 = bf16_hi(xs[e2]);
+    const float y0 = bf16_lo(ys[e2]), y1 = bf16_hi(ys[e2]);
+    xs[e2] = pack_f16_sat(x0 * cs.x - y0 * cs.y, x1 * cs.z - y1 * cs.w);
+    ys[e2] = pack_f16_sat(y0 * cs.x + x0 * cs.y, y1 * cs.z + x1 * cs.w);
+  }
+  *px = make_uint4(xs[0], xs[1], xs[2], xs[3]);
+  *py = make_uint4(ys[0], ys[1], ys[2], ys[3]);
+}
+
 __device__ __forceinline__ void rope_row_tab(uint8_t* row_base, int row, int nun,
                                              const float2* tabrow) {
   const float4* t4 = reinterpret_cast<const float4*>(tabrow);
@@ -397,10 +416,12 @@ __global__ void __launch_bounds__(kSwaThreads, 1)
             if (kpos >= p.krot_from && kpos < p.nk) rope_row(sK, L::R_CHUNK, ring_row, kpos, p.rot_dims, s_invf);
             else if (kpos >= 0 && kpos < p.krot_from) f16_row(sK, L::R_CHUNK, ring_row, p.rot_dims);
           }
-        } else if (ctid < 16) {
-          const int ring_row = (useq % kSwaUnits) * 16 + ctid;
-          if (p0 + ctid < p.nk)   // a block's own keys lie in the chunk: never stored rotated
-            rope_row_tab(smem + L::OFF_K + ring_row * 128, ring_row, nun, tab + ctid * 32);
+        } else if (ctid < 64) {   // the 16 new K rows, one (row, unit pair) per thread
+          const int rr = ctid >> 2, u = ctid & 3;
+          const int ring_row = (useq % kSwaUnits) * 16 + rr;
+          if (u < nun && p0 + rr < p.nk)   // a block's own keys lie in the chunk: never stored rotated
+            rope_unit(smem + L::OFF_K + ring_row * 128, ring_row, nun,
+                      reinterpret_cast<const float4*>(tab + rr * 32), u);
         }
       }
       fence_proxy_async_smem();
