@@ -76,7 +76,7 @@ struct SwaLayout {
   static constexpr int OFF_K = OFF_Q + 2 * Q_STAGE;
   static constexpr int OFF_V = OFF_K + 3 * R_CHUNK;
   static constexpr int OFF_TAB = OFF_V + 2 * R_CHUNK;
-  static constexpr int TAB_BYTES = kSwaP * 32 * 8;     // 16 positions x 32 (cos, sin)
+  static constexpr int TAB_BYTES = kSwaP * 32 * 8;     // 16 positions x 32 frequencies x (cos, sin)
   static constexpr int OFF_MISC = OFF_TAB + 2 * TAB_BYTES;
   static constexpr int MISC_BYTES = 512 + 32 * 8;
   static constexpr int SMEM = OFF_MISC + MISC_BYTES + 1024;
@@ -103,9 +103,31 @@ enum : int {
   kSwNumBars = 50
 };
 
+// (x, y) <- (x cos - y sin, y cos + x sin) for two rotation pairs: xw and yw each hold two
+// bf16 (dims k, k+1 of the first and of the second half), cs = (cos k, cos k+1, sin k,
+// sin k+1). Packed f32x2 arithmetic, results rounded to f16 with clamping.
+__device__ __forceinline__ void rot_pair(uint32_t& xw, uint32_t& yw, const float4 cs) {
+  unsigned long long x, y, c, s, ys, xc, yc, xr, yr;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "r"(xw << 16), "r"(xw & 0xFFFF0000u));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(y) : "r"(yw << 16), "r"(yw & 0xFFFF0000u));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(c) : "f"(cs.x), "f"(cs.y));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(s) : "f"(cs.z), "f"(cs.w));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(ys) : "l"(y), "l"(s));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(xc) : "l"(x), "l"(c));
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(xr) : "l"(xc), "l"(ys));
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(yc) : "l"(y), "l"(c));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(yr) : "l"(x), "l"(s), "l"(yc));
+  float a0, a1, b0, b1;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(xr));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(b0), "=f"(b1) : "l"(yr));
+  xw = pack_f16_sat(a0, a1);
+  yw = pack_f16_sat(b0, b1);
+}
+
 // Rotates dims [0, 16 * nun) (nun <= 4, i.e. rot_dims <= 64, all in the first 64-dim
-// chunk) of one tile row with its (cos, sin) table row. Two unit pairs at a time: loads
-// first, then the math, then the stores, as plain shared-memory accesses.
+// chunk) of one tile row with its table row (float4 per two dims, see rot_pair). Two unit
+// pairs at a time: loads first, then the math, then the stores, as plain shared-memory
+// accesses.
 __device__ __forceinline__ void rope_half(uint8_t* row_base, int row, int nun, const float4* t4,
                                           int ubeg) {
   uint4 x[2], y[2];
@@ -124,13 +146,7 @@ __device__ __forceinline__ void rope_half(uint8_t* row_base, int row, int nun, c
       uint32_t xs[4] = {x[q].x, x[q].y, x[q].z, x[q].w};
       uint32_t ys[4] = {y[q].x, y[q].y, y[q].z, y[q].w};
 #pragma unroll
-      for (int e2 = 0; e2 < 4; ++e2) {
-        const float4 cs = t4[u * 4 + e2];   // (cos k, sin k, cos k+1, sin k+1), k = 8u + 2e2
-        const float x0 = bf16_lo(xs[e2]), x1 = bf16_hi(xs[e2]);
-        const float y0 = bf16_lo(ys[e2]), y1 = bf16_hi(ys[e2]);
-        xs[e2] = pack_f16_sat(x0 * cs.x - y0 * cs.y, x1 * cs.z - y1 * cs.w);
-        ys[e2] = pack_f16_sat(y0 * cs.x + x0 * cs.y, y1 * cs.z + x1 * cs.w);
-      }
+      for (int e2 = 0; e2 < 4; ++e2) rot_pair(xs[e2], ys[e2], t4[u * 4 + e2]);   // k = 8u + 2e2
       *reinterpret_cast<uint4*>(row_base + ((u ^ (row & 7)) << 4)) =
           make_uint4(xs[0], xs[1], xs[2], xs[3]);
       *reinterpret_cast<uint4*>(row_base + (((u + nun) ^ (row & 7)) << 4)) =
@@ -147,20 +163,12 @@ __device__ __forceinline__ void rope_unit(uint8_t* row_base, int row, int nun, c
   uint32_t xs[4] = {x.x, x.y, x.z, x.w};
   uint32_t ys[4] = {y.x, y.y, y.z, y.w};
 #pragma unroll
-  for (int e2 = 0; e2 < 4; ++e2) {
-    const float4 cs = t4[u * 4 + e2];
-    const float x0 = bf16_lo(xs[e2]), x1 = bf16_hi(xs[e2]);
-    const float y0 = bf16_lo(ys[e2]), y1 = bf16_hi(ys[e2]);
-    xs[e2] = pack_f16_sat(x0 * cs.x - y0 * cs.y, x1 * cs.z - y1 * cs.w);
-    ys[e2] = pack_f16_sat(y0 * cs.x + x0 * cs.y, y1 * cs.z + x1 * cs.w);
-  }
+  for (int e2 = 0; e2 < 4; ++e2) rot_pair(xs[e2], ys[e2], t4[u * 4 + e2]);
   *px = make_uint4(xs[0], xs[1], xs[2], xs[3]);
   *py = make_uint4(ys[0], ys[1], ys[2], ys[3]);
 }
 
-__device__ __forceinline__ void rope_row_tab(uint8_t* row_base, int row, int nun,
-                                             const float2* tabrow) {
-  const float4* t4 = reinterpret_cast<const float4*>(tabrow);
+__device__ __forceinline__ void rope_row_tab(uint8_t* row_base, int row, int nun, const float4* t4) {
   rope_half(row_base, row, nun, t4, 0);
   rope_half(row_base, row, nun, t4, 2);
 }
@@ -371,7 +379,7 @@ __global__ void __launch_bounds__(kSwaThreads, 1)
       if (first) seq += 8;
       const int useq = seq++;
       const int p0 = p.q_off + t * kSwaP;            // absolute position of the block
-      float2* tab = reinterpret_cast<float2*>(smem + L::OFF_TAB + (i & 1) * L::TAB_BYTES);
+      float* tab = reinterpret_cast<float*>(smem + L::OFF_TAB + (i & 1) * L::TAB_BYTES);
       if (ctid == 0) SWA_TRACE(i, 0);
       // (cos, sin) of the block's 16 positions (double buffered: tile i - 1 may still read)
       if (half > 0) {
@@ -381,7 +389,9 @@ __global__ void __launch_bounds__(kSwaThreads, 1)
           const double nrev = rint(ang * 0.15915494309189535);
           float sn, cs;
           __sincosf(static_cast<float>(fma(-nrev, 6.283185307179586, ang)), &sn, &cs);
-          tab[pp * 32 + k] = make_float2(cs, sn);
+          float* tk = tab + pp * 64 + (k >> 1) * 4 + (k & 1);   // (cos k, cos k+1, sin k, sin k+1)
+          tk[0] = cs;
+          tk[2] = sn;
         }
         mbar_arrive(bar(kSwTab + (i & 1)));   // (bounded waits only: no hardware named barrier)
         if (!wait_all(bar(kSwTab + (i & 1)), (i >> 1) & 1)) break;
@@ -390,7 +400,7 @@ __global__ void __launch_bounds__(kSwaThreads, 1)
       if (ctid == 0) SWA_TRACE(i, 1);
       if (half > 0 && t * kSwaP + (ctid >> 3) < p.n)
         rope_row_tab(smem + L::OFF_Q + (i & 1) * L::Q_STAGE + ctid * 128, ctid, nun,
-                     tab + (ctid >> 3) * 32);
+                     reinterpret_cast<const float4*>(tab + (ctid >> 3) * 64));
       // K units of this block: the new one, or the whole window at the start of a run
       bool ok = true;
       const int s_first = first ? useq - 8 : useq;
@@ -421,7 +431,7 @@ __global__ void __launch_bounds__(kSwaThreads, 1)
           const int ring_row = (useq % kSwaUnits) * 16 + rr;
           if (u < nun && p0 + rr < p.nk)   // a block's own keys lie in the chunk: never stored rotated
             rope_unit(smem + L::OFF_K + ring_row * 128, ring_row, nun,
-                      reinterpret_cast<const float4*>(tab + rr * 32), u);
+                      reinterpret_cast<const float4*>(tab + rr * 64), u);
         }
       }
       fence_proxy_async_smem();
