@@ -103,6 +103,46 @@ enum : int {
   kSwNumBars = 50
 };
 
+// Packed f32x2 helpers (two fp32 lanes in one 64-bit register pair, rounded per lane).
+// Volatile: its inputs come from tcgen05.ld, so it must stay after the wait::ld that follows
+// the load (volatile asm statements keep their order).
+__device__ __forceinline__ unsigned long long f2_bits(uint32_t lo, uint32_t hi) {
+  unsigned long long r;
+  asm volatile("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+  return r;
+}
+__device__ __forceinline__ unsigned long long f2_pack(float lo, float hi) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 f2_unpack(unsigned long long x) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(x));
+  return r;
+}
+__device__ __forceinline__ unsigned long long f2_fma(unsigned long long a, unsigned long long b,
+                                                     unsigned long long c) {
+  unsigned long long r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ unsigned long long f2_add(unsigned long long a, unsigned long long b) {
+  unsigned long long r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ unsigned long long f2_mul(unsigned long long a, unsigned long long b) {
+  unsigned long long r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float swa_max3(float a, float b, float c) {   // volatile: see f2_bits
+  float r;
+  asm volatile("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // (x, y) <- (x cos - y sin, y cos + x sin) for two rotation pairs: xw and yw each hold two
 // bf16 (dims k, k+1 of the first and of the second half), cs = (cos k, cos k+1, sin k,
 // sin k+1). Packed f32x2 arithmetic, results rounded to f16 with clamping.
@@ -503,9 +543,13 @@ __global__ void __launch_bounds__(kSwaThreads, 1)
         for (int q = 0; q < 2; ++q) {
           float mq = -INFINITY;
           if (k[q] == 2) {
+            float mb = -INFINITY;
 #pragma unroll
-            for (int e = 0; e < 16; e += 2)
-              mq = fmaxf(mq, fmaxf(__uint_as_float(v[q][e]), __uint_as_float(v[q][e + 1])));
+            for (int e = 0; e < 16; e += 4) {
+              mq = swa_max3(mq, __uint_as_float(v[q][e]), __uint_as_float(v[q][e + 1]));
+              mb = swa_max3(mb, __uint_as_float(v[q][e + 2]), __uint_as_float(v[q][e + 3]));
+            }
+            mq = fmaxf(mq, mb);
           } else if (k[q] == 1) {
 #pragma unroll
             for (int e = 0; e < 16; ++e)
@@ -520,26 +564,28 @@ __global__ void __launch_bounds__(kSwaThreads, 1)
       // pass 2: P = exp2(a - amax) (0 outside the window), packed f16 into the S columns
       float sum0 = 0.f, sum1 = 0.f;
       // P of one slot block into pk; returns its sum
+      const unsigned long long sc2 = f2_pack(p.scale_log2, p.scale_log2), nref2 = f2_pack(-ref, -ref);
       auto p_block = [&](const uint32_t (&v)[16], int k, int elo, int ehi, uint32_t (&pk)[8]) -> float {
-        float sa = 0.f, sb = 0.f;
         if (k == 0) {
 #pragma unroll
           for (int e = 0; e < 8; ++e) pk[e] = 0u;
           return 0.f;
         }
+        unsigned long long acc = f2_pack(0.f, 0.f);   // even and odd columns
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          float a0 = ex2(fmaf(__uint_as_float(v[2 * e]), p.scale_log2, -ref));
-          float a1 = ex2(fmaf(__uint_as_float(v[2 * e + 1]), p.scale_log2, -ref));
+          const float2 y = f2_unpack(f2_fma(f2_bits(v[2 * e], v[2 * e + 1]), sc2, nref2));
+          float a0 = ex2(y.x);
+          float a1 = ex2(y.y);
           if (k == 1) {
             a0 = (2 * e >= elo && 2 * e <= ehi) ? a0 : 0.f;
             a1 = (2 * e + 1 >= elo && 2 * e + 1 <= ehi) ? a1 : 0.f;
           }
-          sa += a0;
-          sb += a1;
+          acc = f2_add(acc, f2_pack(a0, a1));
           pk[e] = pack_f16(a0, a1);
         }
-        return sa + sb;
+        const float2 sab = f2_unpack(acc);
+        return sab.x + sab.y;
       };
 #pragma unroll 1
       for (int c = 0; c < kSwaUnits; c += 2) {
@@ -590,12 +636,15 @@ __global__ void __launch_bounds__(kSwaThreads, 1)
           mbar_arrive(bar(kSwTmFree + w));
         }
         if (row_ok) {
+          const unsigned long long il2 = f2_pack(inv_l, inv_l);
 #pragma unroll
           for (int q = 0; q < 2; ++q) {
             uint32_t pk[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e)
-              pk[e] = pack_bf16(__uint_as_float(v[q][2 * e]) * inv_l, __uint_as_float(v[q][2 * e + 1]) * inv_l);
+            for (int e = 0; e < 8; ++e) {
+              const float2 o = f2_unpack(f2_mul(f2_bits(v[q][2 * e], v[q][2 * e + 1]), il2));
+              pk[e] = pack_bf16(o.x, o.y);
+            }
             uint4* dst = reinterpret_cast<uint4*>(orow + (2 * hh + q) * 16);
             dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
             dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);

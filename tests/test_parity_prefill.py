@@ -63,6 +63,30 @@ def test_swa_ring_kernel(cuda_device, B, n, hq, hkv, window, rot):
     _run_and_compare(inp, window, wl.SWA_THETA, rot, cuda_device, f"swa-ring B={B} n={n} W={window}")
 
 
+@pytest.mark.parametrize("B,n,hq,hkv,window,rot,period", [
+    (1, 2000, 16, 2, 128, 64, 400),
+    (2, 1500, 8, 1, 129, 32, 333),
+    (1, 1200, 64, 8, 128, 64, 64),
+])
+def test_swa_ring_kernel_steep_scores(cuda_device, B, n, hq, hkv, window, rot, period):
+    """Scores that climb by ~2.5 (log2 units) per 16 keys inside a window, resetting every
+    `period` keys: the ring kernel's single-pass softmax must move its reference (and scale
+    the P blocks already written) several times per row, and keep it where the row max comes
+    first."""
+    inp = wl.prefill_inputs(B, n, hq, hkv, seed=170 + n + period)
+    # unrotated dims: q += 1, k += 4.7 (t mod period) / period, i.e. about 128 * 4.7 / period
+    # added to every score per key of the saw tooth
+    t = torch.arange(n, dtype=torch.float32)
+    shift = 4.7 * torch.remainder(t, period) / period
+    k = inp["k"].float()
+    k[..., 64:] += shift[None, :, None, None]
+    q = inp["q"].float()
+    q[..., 64:] += 1.0
+    inp["k"], inp["q"] = k.to(torch.bfloat16), q.to(torch.bfloat16)
+    _run_and_compare(inp, window, wl.SWA_THETA, rot, cuda_device,
+                     f"swa-ring steep B={B} n={n} W={window} period={period}")
+
+
 @pytest.mark.parametrize("B,n,hq,hkv,rot,k_scale", [
     (1, 129, 8, 1, 64, 0.5),
     (1, 600, 16, 1, 64, 0.5),         # GA heads 16 per KV head, several key tiles
