@@ -170,6 +170,15 @@ def decode_fp8_inputs(batch, hq, hkv, capacity, lengths, *, seed, device="cpu"):
     return inp
 
 
+def integer_qk(batch, hq, hkv, capacity, *, seed, device="cpu", lo=-2, hi=2):
+    """q [B,Hq,192] and k_cache [B,cap,Hkv,192] bf16 with integer entries uniform in [lo, hi]:
+    every dot product is an integer, exact in fp32 and float64 alike (ties included)."""
+    g = _gen(seed + 17, "cpu")
+    q = torch.randint(lo, hi + 1, (batch, hq, DQK), generator=g).to(torch.bfloat16)
+    k = torch.randint(lo, hi + 1, (batch, capacity, hkv, DQK), generator=g).to(torch.bfloat16)
+    return q.to(device), k.to(device)
+
+
 def sorted_unique_indices(batch, hkv, n_sel, hi_excl, *, seed):
     """[B, Hkv, n_sel] int32, each row sorted unique uniform in [0, hi_excl[b])."""
     g = _gen(seed + 13, "cpu")

@@ -34,3 +34,12 @@ def test_sorted_unique_indices():
 def test_lengths_uniform_range():
     L = wl.lengths_uniform(64, 4096, 131072, seed=1004)
     assert L.dtype == torch.int32 and int(L.min()) >= 4096 and int(L.max()) <= 131072
+
+
+def test_integer_qk_is_seeded_and_small_integers():
+    q, k = wl.integer_qk(2, 8, 2, 50, seed=3)
+    q2, k2 = wl.integer_qk(2, 8, 2, 50, seed=3)
+    assert torch.equal(q, q2) and torch.equal(k, k2)
+    assert q.shape == (2, 8, 192) and k.shape == (2, 50, 2, 192)
+    for t in (q.float(), k.float()):
+        assert torch.equal(t, t.round()) and t.min() >= -2 and t.max() <= 2
