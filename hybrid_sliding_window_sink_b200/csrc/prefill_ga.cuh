@@ -45,6 +45,41 @@ __device__ __forceinline__ uint32_t pack_f16_satfinite(float lo, float hi) {
   return r;
 }
 
+// Packed f32x2 arithmetic (two fp32 lanes per 64-bit register pair, rounded per lane).
+// Volatile: its inputs come from tcgen05.ld, so it stays after the wait::ld that follows the
+// load (volatile asm statements keep their order).
+__device__ __forceinline__ unsigned long long ga_f2_bits(uint32_t lo, uint32_t hi) {
+  unsigned long long r;
+  asm volatile("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+  return r;
+}
+__device__ __forceinline__ unsigned long long ga_f2_pack(float lo, float hi) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 ga_f2_unpack(unsigned long long x) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(x));
+  return r;
+}
+__device__ __forceinline__ unsigned long long ga_f2_fma(unsigned long long a, unsigned long long b,
+                                                        unsigned long long c) {
+  unsigned long long r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ unsigned long long ga_f2_add(unsigned long long a, unsigned long long b) {
+  unsigned long long r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ unsigned long long ga_f2_mul(unsigned long long a, unsigned long long b) {
+  unsigned long long r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
 // 32 consecutive TMEM columns of this warp's 32 lanes.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   tmem_ld16(taddr, *reinterpret_cast<uint32_t(*)[16]>(r));
@@ -495,7 +530,9 @@ __global__ void __launch_bounds__(kGaThreads, 1)
         }
         const float ref = m == -INFINITY ? 0.f : m;
         // pass 2: P = 2^(a - ref) (0 above the diagonal), bf16 into S columns [0, 64)
-        float sa = 0.f, sb = 0.f;
+        const unsigned long long sc2 = ga_f2_pack(p.scale_log2, p.scale_log2);
+        const unsigned long long nref2 = ga_f2_pack(-ref, -ref);
+        unsigned long long sab = ga_f2_pack(0.f, 0.f);   // row sums of even and odd columns
         auto pass2 = [&](auto masked) {
 #pragma unroll 1
           for (int c = 0; c < kGaBN; c += 64) {
@@ -512,14 +549,14 @@ __global__ void __launch_bounds__(kGaThreads, 1)
 #pragma unroll
               for (int e = 0; e < 8; ++e) {
                 const int col = 16 * q + 2 * e;
-                float a0 = ex2(fmaf(__uint_as_float(v[col]), p.scale_log2, -ref));
-                float a1 = ex2(fmaf(__uint_as_float(v[col + 1]), p.scale_log2, -ref));
+                const float2 y = ga_f2_unpack(ga_f2_fma(ga_f2_bits(v[col], v[col + 1]), sc2, nref2));
+                float a0 = ex2(y.x);
+                float a1 = ex2(y.y);
                 if (decltype(masked)::value) {
                   a0 = col <= lim ? a0 : 0.f;
                   a1 = col + 1 <= lim ? a1 : 0.f;
                 }
-                sa += a0;
-                sb += a1;
+                sab = ga_f2_add(sab, ga_f2_pack(a0, a1));
                 pk[e] = pack_bf16(a0, a1);
               }
               tmem_st8(trow + (c >> 1) + 8 * q, pk);
@@ -533,7 +570,8 @@ __global__ void __launch_bounds__(kGaThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(kGaPReady + grp));
-        l += sa + sb;
+        const float2 s2 = ga_f2_unpack(sab);
+        l += s2.x + s2.y;
       }
       if (!ok) break;
       // epilogue after the item's last PV: o = O / l, lse = (m + log2 l) ln 2
@@ -549,10 +587,13 @@ __global__ void __launch_bounds__(kGaThreads, 1)
         tmem_wait_ld();
         if (row_ok) {
           uint32_t pk[16];
+          const unsigned long long il2 = ga_f2_pack(inv_l, inv_l);
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            pk[e] = pack_bf16(__uint_as_float(v0[2 * e]) * inv_l, __uint_as_float(v0[2 * e + 1]) * inv_l);
-            pk[8 + e] = pack_bf16(__uint_as_float(v1[2 * e]) * inv_l, __uint_as_float(v1[2 * e + 1]) * inv_l);
+            const float2 o0 = ga_f2_unpack(ga_f2_mul(ga_f2_bits(v0[2 * e], v0[2 * e + 1]), il2));
+            const float2 o1 = ga_f2_unpack(ga_f2_mul(ga_f2_bits(v1[2 * e], v1[2 * e + 1]), il2));
+            pk[e] = pack_bf16(o0.x, o0.y);
+            pk[8 + e] = pack_bf16(o1.x, o1.y);
           }
           uint4* dst = reinterpret_cast<uint4*>(orow + c * 16);
           dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
