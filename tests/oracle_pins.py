@@ -430,6 +430,15 @@ def check_select_tokens(ref):
     o2, l2 = ref.decode(q, k, v, "linear", L, sink)
     np.testing.assert_allclose(o1, o2, rtol=1e-12, atol=1e-13)
     np.testing.assert_allclose(l1, l2, rtol=0, atol=1e-12)
+    # real-valued scores (distinct almost surely): the kept set is a library top-k of the
+    # group-max logits, computed here with numpy's argpartition on an explicit product
+    qr = r.standard_normal((1, 8, 24))
+    kr = r.standard_normal((1, 300, 2, 24))
+    got = ref.select_tokens(qr, kr, [300], 20, 37)
+    for g in range(2):
+        logits = np.einsum("td,hd->th", kr[0, :280, g], qr[0, 4 * g:4 * g + 4])
+        best = np.argpartition(-logits.max(axis=1), 37)[:37]
+        assert np.array_equal(got[0, g], np.sort(best))
 
 
 def check_e4m3_decoding(ref):

@@ -193,6 +193,7 @@ def test_select_tokens_rejects_before_launch(L):
     assert sel(ws=None) == 5
     assert sel(wsb=16) == 5
     assert sel(q=P(0x10002)) == 4
+    assert sel(n_sel=0) == 0          # nothing to select: OK without a launch
     need = L.mimo_attn_select_workspace_size(ctypes.byref(s), 4096)
     assert need == 1 * 4 * 4096 * 4 + 1 * 4 * 4 * 256 * 2      # keys, then top-byte histograms
     # key rows padded to 16 bytes
