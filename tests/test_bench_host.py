@@ -1,0 +1,84 @@
+"""Host-side arithmetic of bench.py (no GPU): the algorithmic FLOP and byte counts that
+every roofline fraction divides by, and the hash guard on the recorded DRAM traffic."""
+
+import hashlib
+import json
+import os
+
+import pytest
+
+import bench
+from hybrid_sliding_window_sink_b200 import workloads as wl
+
+
+def _pairs_brute(n, window):
+    if window <= 0 or window >= n:
+        return sum(i + 1 for i in range(n))
+    return sum(i - max(0, i - window + 1) + 1 for i in range(n))
+
+
+@pytest.mark.parametrize("n", [1, 5, 130, 300])
+@pytest.mark.parametrize("window", [0, 1, 7, 128, 129, 500])
+def test_swa_pairs_matches_brute_force(n, window):
+    assert bench.swa_pairs(n, window) == _pairs_brute(n, window)
+
+
+def test_headline_prefill_work():
+    """SWA layer, n=32768, 64 Q / 8 KV, W=128: 171.5 GFLOP and 1.518 GB algorithmic."""
+    flops, nbytes = bench.prefill_work(wl.SWA_PREFILL)
+    pairs = 32768 * 128 - 128 * 127 // 2
+    assert flops == 2.0 * (192 + 128) * pairs * 64
+    assert abs(flops / 171.5e9 - 1) < 1e-3
+    q = 32768 * 64 * 192 * 2
+    kv = 32768 * 8 * (192 + 128) * 2
+    o = 32768 * 64 * 128 * 2
+    lse = 64 * 32768 * 4
+    assert nbytes == q + kv + o + lse + 64 * 4
+    assert abs(nbytes / 1.518e9 - 1) < 1e-3
+
+
+def test_decode_byte_counts():
+    hq, hkv = 64, 8
+    ring = bench.decode_layer_bytes([100, 300], hq, hkv, "ring", 128)
+    lin = bench.decode_layer_bytes([100, 300], hq, hkv, "linear", 4096)
+    per_tok = hkv * (192 + 128) * 2
+    assert lin - ring == (300 - 128) * per_tok           # the ring holds only 128 slots
+    # one-token multi-query decode counts exactly what decode counts
+    assert bench.mtp_layer_bytes([100, 300], hq, hkv, "ring", 128, 1) == ring
+    # FP8: 320 B of E4M3 + two fp32 scales per (token, KV head), same q / out / lse
+    fp8 = bench.fp8_decode_layer_bytes([100, 300], hq, hkv, "linear", 4096)
+    assert lin - fp8 == 400 * hkv * (640 - 328)
+
+
+def test_roofline_fields():
+    r = bench.roofline_hbm(6.5578e9, 1.0, {"hbm_gbs": 6557.8}, "measured", traffic=123)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s" and r["traffic"] == 123
+    assert r["achieved"] == 6557.8 and r["frac"] == 1.0
+    t = bench.roofline_tensor(1.6637e12, 1.0, 1663.7, "measured")
+    assert t["bound"] == "tensor" and abs(t["frac"] - 1.0) < 1e-9
+
+
+def test_traffic_reported_only_while_sources_match(tmp_path, monkeypatch):
+    csrc = tmp_path / "hybrid_sliding_window_sink_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "k.cuh").write_text("kernel v1\n")
+    sha = hashlib.sha256(b"kernel v1\n").hexdigest()[:16]
+    (tmp_path / "profiles").mkdir()
+    rec = {"k": {"sources": ["k.cuh"], "sha": sha, "bytes_per_unit": 10.5}}
+    (tmp_path / "profiles" / "traffic.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.traffic_for("k", 4) == 42
+    assert bench.traffic_for("missing", 4) is None
+    (csrc / "k.cuh").write_text("kernel v2\n")             # the kernel changed: no traffic
+    assert bench.traffic_for("k", 4) is None
+
+
+def test_recorded_traffic_files_exist():
+    with open(os.path.join(bench.ROOT, "profiles", "traffic.json")) as f:
+        rec = json.load(f)
+    for key, r in rec.items():
+        if key.startswith("_"):
+            continue
+        assert os.path.exists(os.path.join(bench.ROOT, r["capture"])), key
+        for src in r["sources"]:
+            assert os.path.exists(os.path.join(bench.ROOT, "hybrid_sliding_window_sink_b200", "csrc", src))
