@@ -166,9 +166,11 @@ mimo_status mimo_attn_sparse(const mimo_shape* shape, const void* q, const void*
  *       rot_dims: as mimo_attn_prefill
  *  out  [B, n, Hq, 128] bf16 device; lse [B, Hq, n] fp32 device or NULL
  *
- * Full-causal chunks with 8 or 16 query heads per KV head run on the GA pair kernel, all other
- * shapes (SWA windows included) on the generic prefill kernel. Errors as mimo_attn_prefill;
- * MIMO_ERR_SHAPE also for pos_offset < 0.
+ * Full-causal chunks with 8 or 16 query heads per KV head run on the GA pair kernel; SWA
+ * chunks with 8 query heads per KV head, window <= 129, rot_dims <= 64 and pos_offset a
+ * multiple of 16 on the K/V-ring kernel (the fast path for SWA layers: choose chunk
+ * boundaries on multiples of 16); all other shapes on the generic prefill kernel. Errors as
+ * mimo_attn_prefill; MIMO_ERR_SHAPE also for pos_offset < 0.
  */
 mimo_status mimo_attn_prefill_chunk(const mimo_shape* shape, const void* q, const void* k,
                                     const void* v, int pos_offset, int k_prefix_rotated,
