@@ -82,3 +82,35 @@ def test_recorded_traffic_files_exist():
         assert os.path.exists(os.path.join(bench.ROOT, r["capture"])), key
         for src in r["sources"]:
             assert os.path.exists(os.path.join(bench.ROOT, "hybrid_sliding_window_sink_b200", "csrc", src))
+
+
+def _run_reference(monkeypatch, capsys, rank="0"):
+    monkeypatch.setattr(bench, "oracle_positions_for", lambda case, seconds: 32)
+    monkeypatch.setattr("sys.argv", ["bench.py", "--impl", "reference", "--steps", "2", "--warmup", "3"])
+    monkeypatch.setenv("RANK", rank)
+    monkeypatch.setenv("WORLD_SIZE", "2" if rank != "0" else "1")
+    monkeypatch.setenv("LOCAL_RANK", rank)
+    bench.main()
+    return [l for l in capsys.readouterr().out.splitlines() if l.startswith("{")]
+
+
+def test_reference_arm_json_contract(monkeypatch, capsys):
+    """`bench.py --impl reference` (the float64 oracle on host cores, on a 32-position sample
+    here): one JSON line with the contract's keys, the oracle as its cpu_baseline."""
+    lines = _run_reference(monkeypatch, capsys)
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC
+    assert d["value"] > 0 and d["unit"] == "TFLOP/s" and d["higher_is_better"] is True
+    assert d["steps"] == 2 and d["warmup"] >= 3 and d["ms_per_step"] > 0
+    assert d["n_gpus"] == 1 and d["scaling"] == "weak" and d["vs_baseline"] is None
+    assert d["dtype"] == "f64" and d["data"] == "synthetic"
+    assert d["config"]["workload"] == wl.SWA_PREFILL.name
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_other_ranks_print_nothing(monkeypatch, capsys):
+    assert _run_reference(monkeypatch, capsys, rank="1") == []
