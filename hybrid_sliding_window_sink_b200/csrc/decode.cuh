@@ -90,13 +90,14 @@ __device__ __forceinline__ int dec_unit_keys(const DecodeParams& p, int b, int& 
   return nw + p.n_sel;
 }
 
-// Token (row within the sequence) of key t of unit (b, g).
+// Token (row within the sequence) of key t of unit (b, g); -1 for a selected entry that
+// names no token (the -1 padding of a short selection row), which is a masked key.
 __device__ __forceinline__ int dec_token(const DecodeParams& p, int b, int g, int t, int nw,
                                          int L) {
   if (p.mode != kModeSparse) return t;
   if (t < nw) return L - nw + t;
-  int x = __ldg(p.sel + (static_cast<long long>(b) * p.Hkv + g) * p.n_sel + (t - nw));
-  x = x < 0 ? 0 : x;
+  const int x = __ldg(p.sel + (static_cast<long long>(b) * p.Hkv + g) * p.n_sel + (t - nw));
+  if (x < 0) return -1;
   return x < p.cap - 1 ? x : p.cap - 1;
 }
 
@@ -170,8 +171,9 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
       const int idx = tid + i * kDecThreads;
       const int row = idx / 12, u = idx - row * 12;
       const int key = base + row;
-      const bool ok = key < n_here;
-      const int tok = ok ? token_of(key) : 0;
+      int tok = key < n_here ? token_of(key) : -1;
+      const bool ok = tok >= 0;
+      tok = ok ? tok : 0;
       cp_async16(rK + row * kKRow8 + u * 16, kbase8 + (seq0 + tok) * (krow_stride) + u * 16, ok ? 16u : 0u);
     }
 #pragma unroll
@@ -179,16 +181,18 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
       const int idx = tid + i * kDecThreads;
       const int row = idx >> 3, u = idx & 7;
       const int key = base + row;
-      const bool ok = key < n_here;
-      const int tok = ok ? token_of(key) : 0;
+      int tok = key < n_here ? token_of(key) : -1;
+      const bool ok = tok >= 0;
+      tok = ok ? tok : 0;
       cp_async16(rV + row * kVRow8 + u * 16, vbase8 + (seq0 + tok) * (vrow_stride) + u * 16, ok ? 16u : 0u);
     }
     {                                                             // one scale per thread
       const int row = tid & (kDecSub - 1);
       const bool isv = tid >= kDecSub;
       const int key = base + row;
-      const bool ok = key < n_here;
-      const int tok = ok ? token_of(key) : 0;
+      int tok = key < n_here ? token_of(key) : -1;
+      const bool ok = tok >= 0;
+      tok = ok ? tok : 0;
       const float* src = (isv ? p.v_scale : p.k_scale) + (seq0 + tok) * p.Hkv + g;
       cp_async4(rS + (isv ? kDecSub * 4 : 0) + row * 4, src, ok ? 4u : 0u);
     }
@@ -206,8 +210,9 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
       const int idx = tid + i * kDecThreads;
       const int row = idx / 24, u = idx - row * 24;
       const int key = base + row;
-      const bool ok = key < n_here;
-      const int tok = ok ? token_of(key) : 0;
+      int tok = key < n_here ? token_of(key) : -1;
+      const bool ok = tok >= 0;
+      tok = ok ? tok : 0;
       const __nv_bfloat16* src = kbase + (seq0 + tok) * krow_stride + u * 8;
       cp_async16(sK + row * kKRow + ((u ^ (row & 7)) << 4), src, ok ? 16u : 0u);
     }
@@ -216,8 +221,9 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
       const int idx = tid + i * kDecThreads;
       const int row = idx >> 4, u = idx & 15;
       const int key = base + row;
-      const bool ok = key < n_here;
-      const int tok = ok ? token_of(key) : 0;
+      int tok = key < n_here ? token_of(key) : -1;
+      const bool ok = tok >= 0;
+      tok = ok ? tok : 0;
       const __nv_bfloat16* src = vbase + (seq0 + tok) * vrow_stride + u * 8;
       cp_async16(sV + row * kVRow + ((u ^ (row & 7)) << 4), src, ok ? 16u : 0u);
     }
@@ -326,14 +332,16 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
       }
     }
 
-    // Online softmax (log2 domain); masked keys contribute nothing.
+    // Online softmax (log2 domain); masked keys (past the end, or a selected entry that
+    // names no token) contribute nothing.
     const int keybase = st * kDecSub + warp * 16 + tq * 2;
     float s[2][4];
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const bool ok = keybase + nt * 8 + (e & 1) < n_here;
+        const int key = keybase + nt * 8 + (e & 1);
+        const bool ok = key < n_here && (p.mode != kModeSparse || s_tok[key] >= 0);
         const float ksc = FP8 ? s_ks[keybase - st * kDecSub + nt * 8 + (e & 1)] : 1.f;
         s[nt][e] = ok ? sacc[nt][e] * ksc * p.scale_log2 : -INFINITY;
       }
@@ -491,20 +499,26 @@ __global__ void __launch_bounds__(kDV) decode_combine_kernel(const DecodeParams 
   if (d == 0 && p.lse) p.lse[bh] = Lt > 0.f ? (ref + log2f(Lt)) * 0.6931471805599453f : -INFINITY;
 }
 
-// Debug check of sparse preconditions; one thread per (b, g) row.
+// Debug check of sparse preconditions; one thread per (b, g) row. A valid row is a strictly
+// increasing run of tokens in [0, L - recent) followed by zero or more -1 entries.
 __global__ void check_indices_kernel(const int* lengths, const int* sel, int B, int Hkv, int n_sel,
                                      int recent, int cap, unsigned* violations) {
   const int row = blockIdx.x * blockDim.x + threadIdx.x;
   if (row >= B * Hkv) return;
   const int b = row / Hkv;
   const int L = lengths[b];
-  bool bad = L < 1 || L > cap;
+  bool bad = L < 0 || L > cap;
   const int hi = L - recent;
   const int* s = sel + static_cast<long long>(row) * n_sel;
   int prev = -1;
+  bool padding = false;
   for (int i = 0; i < n_sel && !bad; ++i) {
     const int x = s[i];
-    if (x <= prev || x < 0 || x >= hi) bad = true;
+    if (x == -1) {
+      padding = true;
+      continue;
+    }
+    if (padding || x <= prev || x < 0 || x >= hi) bad = true;
     prev = x;
   }
   if (bad) atomicAdd(violations, 1u);

@@ -111,8 +111,10 @@ mimo_status mimo_attn_prefill(const mimo_shape* shape, const void* q, const void
  *             MIMO_CACHE_LINEAR: slot t holds token t; the query attends [0, L_b)
  *  cache_capacity     slots per sequence (>= 1, <= seq_stride_tokens)
  *  seq_stride_tokens  distance between sequences in tokens
- *  lengths  [B] int32 device: L_b >= 1 tokens so far including the query's own token
- *           (linear: L_b <= cache_capacity; values are clamped to the cache)
+ *  lengths  [B] int32 device: L_b >= 0 tokens so far including the query's own token
+ *           (linear: L_b <= cache_capacity; values are clamped to the cache). L_b = 0 (an
+ *           empty cache) is an empty key set: the formula with an empty sum gives o = 0
+ *           and lse = sink (-inf without a sink)
  *  sink     [Hq] fp32 or NULL
  *  out      [B, Hq, 128] bf16 (written); lse [B, Hq] fp32 or NULL
  *  workspace  device scratch of at least mimo_attn_workspace_size(shape, MIMO_OP_DECODE, cache_kind,
@@ -136,7 +138,9 @@ mimo_status mimo_attn_decode(const mimo_shape* shape, const void* q, const void*
  *  cache_capacity   slots per sequence; lengths and indices are clamped to it
  *  recent           size of the forced recent window (128 on MiMo), >= 0
  *  sel_idx [B, Hkv, n_sel] int32 device: per (sequence, KV head) sorted unique token
- *          indices in [0, L_b - recent), shared by the group's query heads
+ *          indices in [0, L_b - recent), shared by the group's query heads, optionally
+ *          followed by -1 entries that name no token (the padding mimo_attn_select_tokens
+ *          writes when a sequence has fewer candidates than n_sel); a -1 entry is skipped
  *  n_sel            number of selected tokens (1024 on MiMo), >= 0
  *  workspace        at least mimo_attn_workspace_size(shape, MIMO_OP_SPARSE, MIMO_CACHE_LINEAR,
  *                   cache_capacity, recent, n_sel) bytes
@@ -277,7 +281,8 @@ mimo_status mimo_attn_sparse_fp8(const mimo_shape* shape, const void* q, const v
  *  k_cache  [B, seq_stride_tokens, Hkv, 192] bf16 device, linear cache of rotated K
  *  lengths  [B] int32 device (clamped to cache_capacity)
  *  sel_idx  [B, Hkv, n_sel] int32 device (written); rows with fewer than n_sel candidates
- *           hold all of them followed by -1 (a precondition violation for mimo_attn_sparse)
+ *           hold all of them followed by -1, which mimo_attn_sparse skips, so selection
+ *           followed by the sparse decode attends every token of such a sequence
  *  workspace  at least mimo_attn_select_workspace_size(shape, cache_capacity) bytes
  *
  * Two launches: a score pass (1,024 candidates per CTA; q . k on the tensor cores with fp32
@@ -331,9 +336,9 @@ mimo_status mimo_attn_sparse_noalloc(const mimo_shape* shape, const void* q, con
                                      float* lse, void* stream);
 
 /* Debug check of sparse-decode preconditions, on `stream`: counts, into the device
- * word *d_violations (which the caller zeroes first), every (b, g) row whose
- * indices are not strictly increasing, fall outside [0, L_b - recent), or whose
- * L_b is outside [1, cache_capacity]. Never traps. */
+ * word *d_violations (which the caller zeroes first), every (b, g) row that is not a
+ * strictly increasing run of indices in [0, L_b - recent) followed by zero or more -1
+ * entries, or whose L_b is outside [0, cache_capacity]. Never traps. */
 mimo_status mimo_attn_check_indices(const mimo_shape* shape, const int* lengths,
                                     const int* sel_idx, int n_sel, int recent,
                                     int cache_capacity, unsigned int* d_violations,

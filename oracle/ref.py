@@ -51,7 +51,11 @@ Readings where the pages are silent (each also listed in the design notes):
   full-attention layer, no separately trained retrieval module; the scoring rule itself
   is not given): for a sequence and KV head, every token outside the recent window is
   scored by its largest attention logit over the group's query heads; the n_sel best
-  are kept (equal scores: lower index first) and returned in increasing order.
+  are kept (equal scores: lower index first) and returned in increasing order. With
+  fewer candidates than n_sel all of them are kept and the row is padded with -1; a
+  negative index in a sparse key list names no token.
+* Empty key set (a decode query over a cache that holds nothing yet): the §4.4 formula
+  with an empty sum, o = 0 and lse = sink (lse = -inf without a sink).
 * FP8 KV cache (the pages size their KV caches in FP8 but give no scaling scheme):
   K and V bytes are OCP FP8 E4M3 (bias 7, no infinities, S.1111.111 is NaN), each
   (token, KV head) row carries one fp32 scale per tensor, and the cached value is
@@ -162,12 +166,17 @@ def sink_softmax(a, sink: float | None):
 
     m = max(max_j a_j, sink); den = exp(sink - m) + sum_j exp(a_j - m);
     s_j = exp(a_j - m) / den. Returns (s, lse) with lse = m + ln(den).
-    ``sink=None`` drops the sink term (exp(sink) = 0).
+    ``sink=None`` drops the sink term (exp(sink) = 0). An empty row is the
+    formula with an empty sum: den = exp(sink - m) with m = sink, so lse = sink
+    and there are no weights; with no sink either, lse = -inf.
     """
     a = _f64(a)
     m = a.max() if a.size else -math.inf
     if sink is not None:
         m = max(m, float(sink))
+    if m == -math.inf:
+        # no key and no sink: the denominator is an empty sum (reading of an empty key set)
+        return np.zeros_like(a), -math.inf
     e = np.exp(a - m)
     den = e.sum()
     if sink is not None:
@@ -282,10 +291,11 @@ def _cache_rows(kind: str, L: int, capacity: int) -> np.ndarray:
 
     ring (SWA pool of O(W) slots): token p lives in slot p mod capacity, so
     the window W(L-1) occupies slots 0..min(L, capacity)-1; linear (GA pool):
-    slots 0..L-1 hold tokens 0..L-1.
+    slots 0..L-1 hold tokens 0..L-1. L = 0 (nothing cached yet) attends no
+    slot: the key set is empty, so o = 0 and lse = sink (§4.4 with an empty sum).
     """
-    if L < 1:
-        raise ValueError("decode needs at least one cached token")
+    if L < 0:
+        raise ValueError("negative cache length")
     if kind == "ring":
         return np.arange(min(L, capacity), dtype=np.int64)
     if kind == "linear":
@@ -362,10 +372,13 @@ def sparse_key_set(L: int, recent: int, sel) -> np.ndarray:
 
     The most recent ``recent`` tokens {L-recent, ..., L-1} together with the
     selected token indices ``sel`` (drawn from outside the window, so the two
-    parts are disjoint), in one set.
+    parts are disjoint), in one set. Negative entries of ``sel`` name no token:
+    they are the padding ``select_tokens`` writes when a sequence has fewer
+    candidates than n_sel, and they are left out.
     """
     win = np.arange(max(0, L - recent), L, dtype=np.int64)
-    return np.concatenate([win, np.asarray(sel, dtype=np.int64)])
+    sel = np.asarray(sel, dtype=np.int64)
+    return np.concatenate([win, sel[sel >= 0]])
 
 
 def sparse_decode(q, k_cache, v_cache, lengths, recent: int, sel_idx, sink, scale=None):
@@ -430,22 +443,23 @@ def select_tokens(q, k_cache, lengths, recent: int, n_sel: int, scale=None) -> n
     """sel [B, Hkv, n_sel] int64: per sequence b and KV head g, the n_sel tokens t in
     [0, L_b - recent) with the largest score max_{h in group g} (q_h . k_t) * scale, equal
     scores taken in increasing t, listed in increasing t. q: [B, Hq, Dqk] (rotated);
-    k_cache: [B, cap, Hkv, Dqk] linear (rotated K)."""
+    k_cache: [B, cap, Hkv, Dqk] linear (rotated K). A sequence with fewer candidates
+    than n_sel keeps all of them (in increasing t) and fills the rest of its row with -1,
+    which the sparse key set skips."""
     q, kc = _f64(q), _f64(k_cache)
     B, Hq, D = q.shape
     Hkv = kc.shape[2]
     group = Hq // Hkv
     sc = _scale(scale, D)
-    out = np.zeros((B, Hkv, n_sel), dtype=np.int64)
+    out = np.full((B, Hkv, n_sel), -1, dtype=np.int64)
     for b in range(B):
-        hi = int(lengths[b]) - recent
-        if hi < n_sel:
-            raise ValueError("fewer candidate tokens than n_sel")
+        hi = max(0, int(lengths[b]) - recent)
+        keep = min(hi, n_sel)
         for g in range(Hkv):
             logits = (kc[b, :hi, g, :] @ q[b, g * group:(g + 1) * group, :].T) * sc   # [hi, group]
             score = logits.max(axis=1)
             order = sorted(range(hi), key=lambda t: (-score[t], t))
-            out[b, g] = np.sort(np.asarray(order[:n_sel], dtype=np.int64))
+            out[b, g, :keep] = np.sort(np.asarray(order[:keep], dtype=np.int64))
     return out
 
 

@@ -441,6 +441,78 @@ def check_select_tokens(ref):
         assert np.array_equal(got[0, g], np.sort(best))
 
 
+def check_empty_key_set(ref):
+    """A decode query over a cache that holds no token yet (L = 0) has an empty key set.
+    rslog.cc §4.4 with an empty sum leaves only the sink term, so the weights are empty,
+    o = 0 and lse = sink; this equals torch SDPA over the sink alone (one zero-valued
+    extra key, §4.2) and torch.logsumexp of the sink, and the V = 1 closed form
+    o = 1 - exp(sink - lse) gives 0. Without a sink lse = -inf. The other sequences of
+    the batch are unaffected, in ring, linear and sparse decode."""
+    r = _rng(41)
+    B, hq, hkv, d, dv, cap = 3, 4, 2, 16, 8, 24
+    q = r.standard_normal((B, hq, d))
+    kc = r.standard_normal((B, cap, hkv, d))
+    vc = r.standard_normal((B, cap, hkv, dv))
+    sink = r.standard_normal(hq)
+    lengths = [0, 7, 24]
+    # the sink alone through SDPA: one key with K = 0, V = 0 and additive logit sink_h
+    qt = torch.zeros(1, hq, 1, d, dtype=torch.float64)
+    kz = torch.zeros(1, hq, 1, d, dtype=torch.float64)
+    vz = torch.zeros(1, hq, 1, dv, dtype=torch.float64)
+    mask = torch.from_numpy(sink).reshape(1, hq, 1, 1)
+    o_sdpa = F.scaled_dot_product_attention(qt, kz, vz, attn_mask=mask)[0, :, 0].numpy()
+    lse_sdpa = torch.logsumexp(torch.from_numpy(sink)[:, None], dim=1).numpy()
+    for kind in ("ring", "linear"):
+        o, lse = ref.decode(q, kc, vc, kind, lengths, sink)
+        np.testing.assert_array_equal(o[0], o_sdpa)
+        np.testing.assert_array_equal(lse[0], lse_sdpa)
+        o1, l1 = ref.decode(q, kc, np.ones_like(vc), kind, lengths, sink)
+        np.testing.assert_allclose(o1[0, :, 0], 1.0 - np.exp(sink - l1[0]), atol=1e-15)
+        o2, l2 = ref.decode(q[1:], kc[1:], vc[1:], kind, lengths[1:], sink)
+        np.testing.assert_array_equal(o[1:], o2)
+        np.testing.assert_array_equal(lse[1:], l2)
+        o3, l3 = ref.decode(q, kc, vc, kind, lengths, None)
+        assert np.all(o3[0] == 0.0) and np.all(np.isneginf(l3[0]))
+        assert np.all(np.isfinite(l3[1:]))
+    sel = np.full((B, hkv, 3), -1)
+    sel[2] = [[0, 5, 9], [1, 2, 3]]
+    o, lse = ref.sparse_decode(q, kc, vc, [0, 7, 24], 8, sel, sink)
+    np.testing.assert_array_equal(o[0], o_sdpa)
+    np.testing.assert_array_equal(lse[0], lse_sdpa)
+
+
+def check_select_short_rows(ref):
+    """aideepthink.cn §四.3 selects n_sel tokens outside the recent window; a sequence
+    with fewer candidates than that keeps every candidate (brute force: the row is
+    0, 1, ..., hi-1), and the rest of its row is -1, which names no token. So selecting
+    and then running the sparse decode over such a sequence attends the whole cache: it
+    equals the dense decode over the linear cache (also for L <= recent, where nothing is
+    selected and the window alone covers the sequence)."""
+    r = _rng(43)
+    B, Hq, Hkv, D, cap, recent, n_sel = 4, 8, 2, 16, 70, 10, 12
+    q = r.standard_normal((B, Hq, D))
+    k = r.standard_normal((B, cap, Hkv, D))
+    v = r.standard_normal((B, cap, Hkv, 8))
+    sink = r.standard_normal(Hq)
+    lengths = [70, 15, 10, 4]           # 60, 5, 0 and 0 candidates
+    sel = ref.select_tokens(q, k, lengths, recent, n_sel)
+    assert sel.shape == (B, Hkv, n_sel)
+    for b, L in enumerate(lengths):
+        hi = max(0, L - recent)
+        for g in range(Hkv):
+            if hi < n_sel:
+                assert list(sel[b, g, :hi]) == list(range(hi))
+                assert np.all(sel[b, g, hi:] == -1)
+            else:
+                assert np.all(sel[b, g] >= 0) and np.all(np.diff(sel[b, g]) > 0)
+    full = ref.select_tokens(q[:1], k[:1], lengths[:1], recent, n_sel)
+    np.testing.assert_array_equal(sel[:1], full)
+    o1, l1 = ref.sparse_decode(q[1:], k[1:], v[1:], lengths[1:], recent, sel[1:], sink)
+    o2, l2 = ref.decode(q[1:], k[1:], v[1:], "linear", lengths[1:], sink)
+    np.testing.assert_allclose(o1, o2, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(l1, l2, rtol=0, atol=1e-12)
+
+
 def check_e4m3_decoding(ref):
     """OCP FP8 E4M3: every one of the 256 byte patterns decodes as torch.float8_e4m3fn
     does, and the landmarks of the format hold (1.0, the largest 448, the smallest
@@ -578,6 +650,8 @@ ALL_CHECKS = [
     check_multi_decode_matches_prefill,
     check_chunked_prefill_matches_whole,
     check_select_tokens,
+    check_select_short_rows,
+    check_empty_key_set,
     check_sparse_membership,
     check_e4m3_decoding,
     check_fp8_decode_reduces_to_bf16,

@@ -56,8 +56,18 @@ MUTANTS = {
     "selection ties to the higher index": ("            order = sorted(range(hi), key=lambda t: (-score[t], t))\n",
                                            "            order = sorted(range(hi), key=lambda t: (-score[t], -t))\n"),
     "selection by the group's mean logit": ("            score = logits.max(axis=1)\n", "            score = logits.mean(axis=1)\n"),
-    "selection reaches into the window": ("        hi = int(lengths[b]) - recent\n        if hi < n_sel:",
-                                          "        hi = int(lengths[b]) - recent + 1\n        if hi < n_sel:"),
+    "selection reaches into the window": ("        hi = max(0, int(lengths[b]) - recent)\n",
+                                          "        hi = max(0, int(lengths[b]) - recent + 1)\n"),
+    "selection pads short rows with token 0": ("    out = np.full((B, Hkv, n_sel), -1, dtype=np.int64)\n",
+                                               "    out = np.zeros((B, Hkv, n_sel), dtype=np.int64)\n"),
+    "selection of a short row drops its last candidate": ("        keep = min(hi, n_sel)\n",
+                                                          "        keep = min(hi - 1, n_sel) if hi < n_sel else n_sel\n"),
+    "sparse key set keeps the -1 padding": ("    return np.concatenate([win, sel[sel >= 0]])",
+                                            "    return np.concatenate([win, sel])"),
+    "empty cache attends slot 0": ("    if L < 0:\n        raise ValueError(\"negative cache length\")\n",
+                                   "    L = max(L, 1)\n"),
+    "empty key set without the sink": ("    m = a.max() if a.size else -math.inf\n",
+                                       "    if not a.size:\n        return np.zeros_like(a), -math.inf\n    m = a.max()\n"),
     "e4m3 exponent bias 8": ("np.exp2(e.astype(np.float64) - 7.0)", "np.exp2(e.astype(np.float64) - 8.0)"),
     "e4m3 subnormal scale": ("m / 8.0 * 2.0 ** -6", "m / 8.0 * 2.0 ** -7"),
     "e4m3 without NaN": ("np.where((e == 15) & (m == 7), np.nan, val)", "val"),

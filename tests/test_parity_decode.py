@@ -94,3 +94,17 @@ def test_decode_deterministic(cuda_device):
     b = _lib.decode(inp["q"], inp["k_cache"], inp["v_cache"], inp["lengths"], inp["sink"], kind="linear")
     torch.cuda.synchronize()
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+@pytest.mark.parametrize("kind,cap,lengths,sink", [
+    ("ring", 128, [0, 1, 200, 0], True),
+    ("ring", 128, [0, 77], False),
+    ("linear", 4000, [0, 4000, 1, 2500], True),     # several chunks per sequence, one empty
+    ("linear", 300, [0, 0, 300], False),
+])
+def test_empty_cache_against_oracle(cuda_device, kind, cap, lengths, sink):
+    """L = 0 (nothing cached yet) is an empty key set: o = 0 and lse = sink, or -inf
+    without a sink, while the other sequences of the batch are unaffected."""
+    inp = wl.decode_inputs(len(lengths), 64, 4 if kind == "linear" else 8, cap, lengths,
+                           seed=330 + cap + len(lengths))
+    _check(inp, kind, cap, cuda_device, f"{kind} with empty caches", sink=sink)

@@ -38,14 +38,45 @@ def test_select_exact_on_integer_scores(cuda_device, B, hq, hkv, cap, lengths, r
     assert np.array_equal(sel.cpu().numpy().astype(np.int64), want)
 
 
-def test_select_too_few_candidates_pads(cuda_device):
-    q, k = _int_inputs(1, 8, 2, 200, seed=5)
+@pytest.mark.parametrize("lengths", [[140, 2000, 128, 0], [129, 1153]])
+def test_select_short_rows_against_oracle(cuda_device, lengths):
+    """Sequences with fewer candidates than n_sel keep all of them, then -1 (the oracle's
+    rule), next to sequences with enough candidates."""
+    B, cap = len(lengths), max(lengths)
+    q, k = _int_inputs(B, 16, 2, cap, seed=5 + cap)
     sel = _lib.select_tokens(q.to(cuda_device), k.to(cuda_device),
-                             torch.tensor([140], dtype=torch.int32, device=cuda_device), recent=128, n_sel=20)
+                             torch.tensor(lengths, dtype=torch.int32, device=cuda_device),
+                             recent=128, n_sel=20)
     torch.cuda.synchronize()
-    s = sel.cpu().numpy()
-    assert np.array_equal(s[0, :, :12], np.tile(np.arange(12), (2, 1)))
-    assert np.all(s[0, :, 12:] == -1)
+    want = ref.select_tokens(wl.to_f64(q), wl.to_f64(k), lengths, 128, 20)
+    assert np.array_equal(sel.cpu().numpy().astype(np.int64), want)
+
+
+def test_select_then_sparse_short_sequences(cuda_device):
+    """Select, then sparse decode, on a batch where some sequences have fewer candidates than
+    n_sel (their rows end in -1): the sparse decode skips the padding and matches the oracle,
+    which here equals the dense decode of those sequences."""
+    B, hq, hkv, cap, recent, n_sel = 4, 64, 4, 3000, 128, 1024
+    lengths = [3000, 700, 128, 5]
+    q, k = _int_inputs(B, hq, hkv, cap, seed=9)
+    d = wl.decode_inputs(B, hq, hkv, cap, lengths, seed=10)
+    dev = cuda_device
+    L = d["lengths"].to(dev)
+    sel = _lib.select_tokens(q.to(dev), k.to(dev), L, recent=recent, n_sel=n_sel)
+    out, lse = _lib.sparse(d["q"].to(dev), k.to(dev), d["v_cache"].to(dev), L, sel, d["sink"].to(dev),
+                           recent=recent)
+    assert _lib.check_indices(L, sel, hq=hq, recent=recent, capacity=cap) == 0
+    torch.cuda.synchronize()
+    assert _lib.last_device_error() == 0
+    want_sel = ref.select_tokens(wl.to_f64(q), wl.to_f64(k), lengths, recent, n_sel)
+    assert np.array_equal(sel.cpu().numpy().astype(np.int64), want_sel)
+    o_ref, l_ref = ref.sparse_decode(wl.to_f64(d["q"]), wl.to_f64(k), wl.to_f64(d["v_cache"]), lengths,
+                                     recent, want_sel, wl.to_f64(d["sink"]))
+    from parity_util import compare
+    compare(wl.to_f64(out), o_ref, wl.to_f64(lse), l_ref, "select -> sparse, short sequences")
+    o_d, l_d = ref.decode(wl.to_f64(d["q"][1:]), wl.to_f64(k[1:]), wl.to_f64(d["v_cache"][1:]), "linear",
+                          lengths[1:], wl.to_f64(d["sink"]))
+    compare(wl.to_f64(out[1:]), o_d, wl.to_f64(lse[1:]), l_d, "short sequences = dense decode")
 
 
 def test_select_random_scores_within_rounding(cuda_device):

@@ -126,12 +126,44 @@ def test_index_membership_bit_exact(cuda_device):
         assert have == want, (h, sorted(have ^ want))
 
 
+def test_sparse_padding_and_empty_cache(cuda_device):
+    """Rows padded with -1 (fewer selected tokens than n_sel) and an empty cache (L = 0):
+    the padding names no token and L = 0 gives o = 0, lse = sink, as the oracle says."""
+    B, hq, hkv, cap, recent, n_sel = 4, 64, 4, 2048, 128, 300
+    lengths = [2048, 300, 0, 129]
+    inp = wl.decode_inputs(B, hq, hkv, cap, lengths, seed=450)
+    sel = np.full((B, hkv, n_sel), -1, dtype=np.int32)
+    r = np.random.default_rng(450)
+    for b, L in enumerate(lengths):
+        hi = max(0, L - recent)
+        for g in range(hkv):
+            m = min(hi, n_sel - 7 * g)     # a different number of real entries per row
+            sel[b, g, :m] = np.sort(r.choice(hi, m, replace=False))
+    inp["sel"] = torch.from_numpy(sel)
+    out, lse = _run(inp, recent, cuda_device)
+    torch.cuda.synchronize()
+    assert _lib.last_device_error() == 0
+    assert _lib.check_indices(inp["lengths"].to(cuda_device), inp["sel"].to(cuda_device), hq=hq,
+                              recent=recent, capacity=cap) == 0
+    o_ref, l_ref = ref.sparse_decode(wl.to_f64(inp["q"]), wl.to_f64(inp["k_cache"]),
+                                     wl.to_f64(inp["v_cache"]), lengths, recent, sel,
+                                     wl.to_f64(inp["sink"]))
+    compare(wl.to_f64(out), o_ref, wl.to_f64(lse), l_ref, "sparse with -1 padding and L = 0")
+
+
 def test_check_indices_counts_violations(cuda_device):
     L = torch.tensor([500, 500, 0], dtype=torch.int32, device=cuda_device)
     good = np.arange(0, 300, 3, dtype=np.int32)
     sel = np.stack([good, good, good, good[::-1].copy(), good, good])
     sel[4, 5] = sel[4, 4]                    # duplicate
     sel = torch.from_numpy(sel.reshape(3, 2, -1)).to(cuda_device)
-    # rows: (0,0) ok, (0,1) ok, (1,0) ok, (1,1) unsorted, (2,*) L=0 -> bad, and (2,0) dup
+    # rows: (0,0) ok, (0,1) ok, (1,0) ok, (1,1) unsorted, (2,*) indices beyond L - recent
+    # (L = 0 itself is allowed), and (2,0) also a duplicate
     n = _lib.check_indices(L, sel, hq=4, recent=128, capacity=1000)
     assert n == 3
+    # -1 padding after the real entries is valid; a -1 before a real entry is not
+    pad = sel.clone()
+    pad[0, 0, 50:] = -1
+    pad[0, 1, 10:20] = -1
+    n2 = _lib.check_indices(L, pad, hq=4, recent=128, capacity=1000)
+    assert n2 == 4
