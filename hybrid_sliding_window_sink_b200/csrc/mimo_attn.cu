@@ -37,7 +37,6 @@ using mimo::PrefillParams;
 
 constexpr int kMaxDevices = 64;
 std::atomic<int> g_sm_count[kMaxDevices];
-std::atomic<unsigned*> g_err_ptr[kMaxDevices];
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
@@ -64,17 +63,60 @@ int sm_count_for(int dev) {
   return n;
 }
 
-unsigned* device_error_ptr(int dev) {
+// Unique ID of the calling thread's current CUDA context (0 when there is none). IDs are
+// never reused within a process, so a context created after a device reset gets a new one.
+unsigned long long current_context_id() {
+  using GetCurrent = CUresult (*)(CUcontext*);
+  using GetId = CUresult (*)(CUcontext, unsigned long long*);
+  static GetCurrent get_current = nullptr;
+  static GetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrent>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetId>(p);
+    cudaGetLastError();
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current && get_id && get_current(&ctx) == CUDA_SUCCESS && ctx) get_id(ctx, &id);
+  return id;
+}
+
+// Device address of a __device__ variable, looked up with cudaGetSymbolAddress once per
+// (device, context) and cached: on the host the symbol names a stand-in, not device memory,
+// and a context created after a device reset may place the module's variables elsewhere.
+struct SymbolAddressCache {
+  std::mutex mu;
+  unsigned long long ctx_id[kMaxDevices] = {};
+  void* addr[kMaxDevices] = {};
+};
+
+template <typename T>
+void* cached_symbol_address(SymbolAddressCache& c, const T& symbol, int dev) {
   if (dev < 0 || dev >= kMaxDevices) return nullptr;
-  unsigned* p = g_err_ptr[dev].load(std::memory_order_acquire);
-  if (p) return p;
+  std::lock_guard<std::mutex> lock(c.mu);
+  const unsigned long long id = current_context_id();
+  if (c.addr[dev] && id != 0 && c.ctx_id[dev] == id) return c.addr[dev];
   void* addr = nullptr;
-  if (cudaGetSymbolAddress(&addr, mimo::g_device_error) != cudaSuccess) {
+  if (cudaGetSymbolAddress(&addr, symbol) != cudaSuccess || addr == nullptr) {
     cudaGetLastError();
     return nullptr;
   }
-  g_err_ptr[dev].store(static_cast<unsigned*>(addr), std::memory_order_release);
-  return static_cast<unsigned*>(addr);
+  c.addr[dev] = addr;
+  c.ctx_id[dev] = current_context_id();   // the lookup made the primary context current
+  return addr;
+}
+
+SymbolAddressCache g_err_cache;
+
+unsigned* device_error_ptr(int dev) {
+  return static_cast<unsigned*>(cached_symbol_address(g_err_cache, mimo::g_device_error, dev));
 }
 
 bool group_ok(int g) { return g == 1 || g == 2 || g == 4 || g == 8 || g == 16; }
@@ -812,23 +854,14 @@ int mimo_attn_version(void) { return 100; }
 // The split-KV partials of mimo_attn_sparse_noalloc live in this library-owned array
 // instead of a caller workspace. Host code must not pass the symbol itself to a kernel:
 // on the host it names a stand-in, not device memory. The device address is looked up
-// once per device (with that device current) and cached.
+// with cudaGetSymbolAddress (that device current) once per device and context, and cached.
 static __device__ __align__(256) unsigned char g_sparse_noalloc_scratch[MIMO_SPARSE_NOALLOC_SCRATCH_BYTES];
 
 namespace {
-std::atomic<void*> g_noalloc_ptr[kMaxDevices];
+SymbolAddressCache g_noalloc_cache;
 
 void* noalloc_scratch(int dev) {
-  if (dev < 0 || dev >= kMaxDevices) return nullptr;
-  void* p = g_noalloc_ptr[dev].load(std::memory_order_acquire);
-  if (p) return p;
-  void* addr = nullptr;
-  if (cudaGetSymbolAddress(&addr, g_sparse_noalloc_scratch) != cudaSuccess || addr == nullptr) {
-    cudaGetLastError();
-    return nullptr;
-  }
-  g_noalloc_ptr[dev].store(addr, std::memory_order_release);
-  return addr;
+  return cached_symbol_address(g_noalloc_cache, g_sparse_noalloc_scratch, dev);
 }
 }  // namespace
 

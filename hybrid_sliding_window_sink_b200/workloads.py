@@ -172,11 +172,33 @@ def decode_fp8_inputs(batch, hq, hkv, capacity, lengths, *, seed, device="cpu"):
 
 def integer_qk(batch, hq, hkv, capacity, *, seed, device="cpu", lo=-2, hi=2):
     """q [B,Hq,192] and k_cache [B,cap,Hkv,192] bf16 with integer entries uniform in [lo, hi]:
-    every dot product is an integer, exact in fp32 and float64 alike (ties included)."""
-    g = _gen(seed + 17, "cpu")
-    q = torch.randint(lo, hi + 1, (batch, hq, DQK), generator=g).to(torch.bfloat16)
-    k = torch.randint(lo, hi + 1, (batch, capacity, hkv, DQK), generator=g).to(torch.bfloat16)
-    return q.to(device), k.to(device)
+    every dot product is an integer, exact in fp32 and float64 alike (ties included).
+    Drawn on ``device`` (a CUDA device avoids a host copy of a large cache)."""
+    g = _gen(seed + 17, device)
+    q = torch.randint(lo, hi + 1, (batch, hq, DQK), generator=g, device=device).to(torch.bfloat16)
+    k = torch.randint(lo, hi + 1, (batch, capacity, hkv, DQK), generator=g,
+                      device=device, dtype=torch.int8).to(torch.bfloat16)
+    return q, k
+
+
+def random_e4m3(shape, g, device):
+    """Uniformly random E4M3 bytes with the two NaN patterns replaced by 0 (a cache holds
+    no NaN), drawn with generator ``g`` on ``device``."""
+    b = torch.randint(0, 256, shape, generator=g, device=device, dtype=torch.int32)
+    b = torch.where((b & 0x7F) == 0x7F, torch.zeros_like(b), b)
+    return b.to(torch.uint8)
+
+
+def random_fp8_cache(batch, capacity, hkv, *, seed, device="cpu", scale_lo=0.002, scale_hi=0.01):
+    """An FP8 KV cache drawn directly as bytes (no bf16 source): k8 [B,cap,Hkv,192] and
+    v8 [B,cap,Hkv,128] random E4M3 bytes, k_scale / v_scale [B,cap,Hkv] fp32 uniform in
+    [scale_lo, scale_hi]. Draw order: k8, v8, k_scale, v_scale."""
+    g = _gen(seed, device)
+    k8 = random_e4m3((batch, capacity, hkv, DQK), g, device)
+    v8 = random_e4m3((batch, capacity, hkv, DV), g, device)
+    ks = torch.empty(batch, capacity, hkv, device=device).uniform_(scale_lo, scale_hi, generator=g)
+    vs = torch.empty(batch, capacity, hkv, device=device).uniform_(scale_lo, scale_hi, generator=g)
+    return k8, v8, ks, vs
 
 
 def sorted_unique_indices(batch, hkv, n_sel, hi_excl, *, seed):

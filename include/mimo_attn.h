@@ -322,9 +322,10 @@ size_t mimo_attn_workspace_size(const mimo_shape* shape, int op, int cache_kind,
  * Arguments and results are those of mimo_attn_sparse without workspace. Returns
  * MIMO_ERR_WORKSPACE, with nothing launched, when these sizes need more scratch than
  * the array holds (mimo_attn_workspace_size(shape, MIMO_OP_SPARSE, ...) larger than
- * MIMO_SPARSE_NOALLOC_SCRATCH_BYTES). The first call on a device looks up the array's
- * device address with that device current (a host-side query, no allocation); make that
- * first call before any stream capture. All calls share the one array: two calls whose
+ * MIMO_SPARSE_NOALLOC_SCRATCH_BYTES). The first call on a device, and the first after a
+ * device reset (a new CUDA context), looks up the array's device address with that device
+ * current (a host-side query, no allocation); make that first call before any stream
+ * capture. All calls share the one array: two calls whose
  * kernels overlap on the GPU (different streams, no ordering between them) race on it
  * and give wrong results; order them on one stream. No part of the array needs to start
  * at zero: each call writes every partial it later reads.

@@ -468,7 +468,7 @@ def select_tokens(q, k_cache, lengths, recent: int, n_sel: int, scale=None) -> n
 # --------------------------------------------------------------------------
 
 def prefill_chunk(q, k, v, pos_offset: int, k_prefix_rotated: bool, sink, window: int,
-                  rope_theta: float, rot_dims: int, scale: float | None = None):
+                  rope_theta: float, rot_dims: int, scale: float | None = None, rows=None):
     """Sink attention of a chunk of n query tokens at positions off .. off+n-1.
 
     q: [B, n, Hq, Dqk] (un-rotated); k: [B, off+n, Hkv, Dqk], v: [B, off+n, Hkv, Dv] hold
@@ -476,7 +476,8 @@ def prefill_chunk(q, k, v, pos_offset: int, k_prefix_rotated: bool, sink, window
     ``k_prefix_rotated`` (a cache holds rotated K) and rotated otherwise; the chunk's key
     rows (positions >= off) are rotated. Query i of the chunk is rotated at position
     off + i and attends window_keys(off + i, window, off + n).
-    Returns (o [B, n, Hq, Dv], lse [B, Hq, n]).
+    Returns (o [B, n, Hq, Dv], lse [B, Hq, n]); with ``rows``, an iterable of (b, h, i)
+    (i counted within the chunk), only those rows: (o [len, Dv], lse [len]) in that order.
     """
     q, k, v = _f64(q), _f64(k), _f64(v)
     B, n, Hq, D = q.shape
@@ -490,6 +491,18 @@ def prefill_chunk(q, k, v, pos_offset: int, k_prefix_rotated: bool, sink, window
     kr = np.stack([rope(k[b], kpos, rope_theta, rot_dims) for b in range(B)])
     if k_prefix_rotated:
         kr[:, :off] = k[:, :off]
+    if rows is not None:
+        rows = list(rows)
+        o = np.zeros((len(rows), v.shape[-1]))
+        lse = np.zeros(len(rows))
+        for r, (b, h, i) in enumerate(rows):
+            g = h // group
+            qrow = rope(q[b, i:i + 1, h:h + 1], np.array([off + i], dtype=np.float64),
+                        rope_theta, rot_dims)[0, 0]
+            keys = window_keys(off + i, window, nk)
+            o[r], lse[r] = attend_row(qrow, kr[b, :, g, :], v[b, :, g, :], keys,
+                                      None if sink is None else float(_f64(sink)[h]), sc)
+        return o, lse
     qpos = off + np.arange(n, dtype=np.float64)
     qr = np.stack([rope(q[b], qpos, rope_theta, rot_dims) for b in range(B)])
     o = np.zeros((B, n, Hq, v.shape[-1]))

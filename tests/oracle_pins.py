@@ -365,6 +365,13 @@ def check_chunked_prefill_matches_whole(ref):
                     o, l = ref.prefill_chunk(q[:, a:b], kk, v[:, :b], a, rotated, sink, window, 1e4, 8)
                     np.testing.assert_allclose(o, o_full[:, a:b], rtol=1e-11, atol=1e-12)
                     np.testing.assert_allclose(l, l_full[:, :, a:b], rtol=0, atol=1e-11)
+                    # the row-sampled form gives exactly the full form's rows
+                    rows = [(0, h, i) for i in sorted({0, (b - a) // 2, b - a - 1}) for h in (0, 3)]
+                    o_r, l_r = ref.prefill_chunk(q[:, a:b], kk, v[:, :b], a, rotated, sink, window,
+                                                 1e4, 8, rows=rows)
+                    for r, (_, h, i) in enumerate(rows):
+                        np.testing.assert_array_equal(o_r[r], o[0, i, h])
+                        assert l_r[r] == l[0, h, i]
     # cache write-back: chunks appended to a ring of 12 slots and to a linear cache
     for kind, cap in (("ring", 12), ("linear", 64)):
         kc = np.zeros((1, cap, hkv, d))

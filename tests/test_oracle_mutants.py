@@ -46,6 +46,9 @@ MUTANTS = {
                                                   "    qpos = np.arange(n, dtype=np.float64)\n"),
     "chunk window measured on the chunk only": ("                keys = window_keys(off + i, window, nk)\n",
                                                 "                keys = window_keys(off + i, window, nk)[-(i + 1):]\n"),
+    "sampled chunk rows at chunk-relative positions": (
+        "            qrow = rope(q[b, i:i + 1, h:h + 1], np.array([off + i], dtype=np.float64),\n",
+        "            qrow = rope(q[b, i:i + 1, h:h + 1], np.array([i], dtype=np.float64),\n"),
     "cached prefix rotated twice": ("    if k_prefix_rotated:\n        kr[:, :off] = k[:, :off]\n",
                                     "    if False:\n        kr[:, :off] = k[:, :off]\n"),
     "appended K left un-rotated": ("            kc[b, slot] = kr[i]\n", "            kc[b, slot] = kn[b, i]\n"),

@@ -101,22 +101,31 @@ def test_cache_append(cuda_device, kind, cap, off, n):
 
 
 def test_append_then_decode_matches_prefill(cuda_device):
-    """Prefill a prompt in two chunks, append both to a ring and a linear cache, then the
-    decode of the last prompt token (as the next step would see it) equals the prefill row."""
+    """Append a prompt to a ring cache in two chunks, then decode the last prompt token as
+    the next step would see it. The oracle side appends with ref.cache_append and stores
+    the values as bf16 (what the cache holds), then runs ref.decode; the GPU's decode also
+    agrees with its own prefill row of that token."""
     n, hq, hkv = 400, 64, 8
     inp = wl.prefill_inputs(1, n, hq, hkv, seed=1600, device=cuda_device)
     whole, lw = _lib.prefill(inp["q"], inp["k"], inp["v"], inp["sink"], window=128,
                              rope_theta=1e4, rot_dims=64)
     ring_k = torch.zeros(1, 128, hkv, 192, dtype=torch.bfloat16, device=cuda_device)
     ring_v = torch.zeros(1, 128, hkv, 128, dtype=torch.bfloat16, device=cuda_device)
+    kc_ref, vc_ref = np.zeros((1, 128, hkv, 192)), np.zeros((1, 128, hkv, 128))
     for a, b in ((0, 333), (333, 400)):
         _lib.cache_append(inp["k"][:, a:b].contiguous(), inp["v"][:, a:b].contiguous(), ring_k, ring_v,
                           pos_offset=a, rope_theta=1e4, rot_dims=64, kind="ring")
-    # the decode query is the rotated q of position n-1 (rotate with the oracle, round to bf16)
+        kc_ref, vc_ref = ref.cache_append(wl.to_f64(inp["k"][:, a:b]), wl.to_f64(inp["v"][:, a:b]), a,
+                                          1e4, 64, "ring", kc_ref, vc_ref)
+    as_bf16 = lambda x: torch.from_numpy(x).to(torch.bfloat16)  # noqa: E731
+    # the decode query is the rotated q of position n-1 (rotated by the oracle, held as bf16)
     qr = ref.rope(wl.to_f64(inp["q"][0, n - 1:n]), np.array([n - 1.0]), 1e4, 64)
-    qd = torch.from_numpy(qr).to(torch.bfloat16).to(cuda_device)
-    o, l = _lib.decode(qd, ring_k, ring_v, torch.tensor([n], dtype=torch.int32, device=cuda_device),
-                       inp["sink"], kind="ring")
+    qd = as_bf16(qr)
+    o, l = _lib.decode(qd.to(cuda_device), ring_k, ring_v,
+                       torch.tensor([n], dtype=torch.int32, device=cuda_device), inp["sink"], kind="ring")
     torch.cuda.synchronize()
+    o_ref, l_ref = ref.decode(wl.to_f64(qd), wl.to_f64(as_bf16(kc_ref)), wl.to_f64(as_bf16(vc_ref)), "ring",
+                              [n], wl.to_f64(inp["sink"]))
+    compare(wl.to_f64(o), o_ref, wl.to_f64(l), l_ref, "append + decode vs oracle")
     compare(wl.to_f64(o[0]), wl.to_f64(whole[0, n - 1]), wl.to_f64(l[0]), wl.to_f64(lw[0, :, n - 1]),
             "append + decode vs prefill row")

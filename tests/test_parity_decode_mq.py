@@ -60,4 +60,8 @@ def test_one_token_matches_decode(cuda_device):
     b, lb = _lib.decode(inp["q_mq"][:, 0].contiguous(), inp["k_cache"], inp["v_cache"], inp["lengths"],
                         inp["sink"], kind="ring")
     torch.cuda.synchronize()
+    o_ref, l_ref = ref.decode(wl.to_f64(inp["q_mq"][:, 0]), wl.to_f64(inp["k_cache"]),
+                              wl.to_f64(inp["v_cache"]), "ring", lengths, wl.to_f64(inp["sink"]))
+    compare(wl.to_f64(a[:, 0]), o_ref, wl.to_f64(la[:, 0]), l_ref, "mq T=1 vs oracle decode")
+    compare(wl.to_f64(b), o_ref, wl.to_f64(lb), l_ref, "decode vs oracle")
     compare(wl.to_f64(a[:, 0]), wl.to_f64(b), wl.to_f64(la[:, 0]), wl.to_f64(lb), "mq T=1 vs decode")

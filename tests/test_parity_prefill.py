@@ -177,22 +177,28 @@ def test_deterministic_and_guarded(cuda_device):
     assert bool((l_buf[:guard] == 7.0).all()) and bool((l_buf[-guard:] == 7.0).all())
 
 
-def _sample_rows(n, nrand, seed, tile_rows=(16, 8)):
+def _sample_rows(n, nrand, seed, ends=256):
+    """The first and last ``ends`` rows, rows around the window and tile boundaries
+    (127/128/129, 143-145, 255/256) and at 64 multiples of 16 spread over the sequence,
+    and ``nrand`` seeded random rows."""
     r = np.random.default_rng(seed)
-    rows = set(range(0, 96)) | set(range(n - 96, n))
+    rows = set(range(0, ends)) | set(range(n - ends, n))
     for t in (127, 128, 129, 143, 144, 145, 255, 256):
         rows |= {t - 1, t, t + 1}
+    rows |= {16 * k for k in range(1, n // 16, max(1, n // (16 * 64)))}
     rows |= set(r.choice(n, nrand, replace=False).tolist())
     return sorted(x for x in rows if 0 <= x < n)
 
 
 @pytest.mark.parametrize("case,nrand,heads", [
-    (wl.SWA_PREFILL, 256, None),
-    (wl.GA_PREFILL, 24, 16),
+    (wl.SWA_PREFILL, 1024, None),
+    (wl.GA_PREFILL, 1024, 4),
 ])
 def test_full_size_sampled(cuda_device, case, nrand, heads):
     """Full-size configurations, exactly as the benchmark launches them, against the
-    oracle on sampled rows (start, end, tile boundaries, seeded random rows)."""
+    oracle on sampled rows: the first and last 256 rows, window and tile boundaries and
+    1,024 seeded random rows. SWA: all 64 heads of every sampled row; GA: 4 heads per row
+    (one per KV head), rotating so that every head is checked on a quarter of the rows."""
     inp = wl.case_prefill_inputs(case, device=cuda_device)
     out, lse = _lib.prefill(inp["q"], inp["k"], inp["v"], inp["sink"], window=case.window,
                             rope_theta=case.theta, rot_dims=wl.ROT_DIMS)
@@ -200,19 +206,22 @@ def test_full_size_sampled(cuda_device, case, nrand, heads):
     assert _lib.last_device_error() == 0
     n = case.seqlen
     pos = _sample_rows(n, nrand, case.seed)
-    hs = list(range(case.hq)) if heads is None else sorted(
-        np.random.default_rng(case.seed + 1).choice(case.hq, heads, replace=False).tolist())
+    G = case.hq // case.hkv
+    if heads is None:
+        head_sets = [list(range(case.hq))] * len(pos)
+    else:   # one head per KV head, shifted by one within the group from row to row
+        head_sets = [[g * G + (a + g) % G for g in range(case.hkv)] for a in range(len(pos))]
     # the oracle receives the exact bf16 values: the sampled query rows and all of K, V
     qs = wl.to_f64(inp["q"][0, pos])                                  # [len(pos), Hq, 192]
-    rows = [(0, h, i) for i in pos for h in hs]
-    q_rows = np.stack([qs[a, h] for a in range(len(pos)) for h in hs])
+    rows = [(0, h, i) for a, i in enumerate(pos) for h in head_sets[a]]
+    q_rows = np.stack([qs[a, h] for a in range(len(pos)) for h in head_sets[a]])
     o_ref, l_ref = ref.prefill_rows(q_rows, wl.to_f64(inp["k"]), wl.to_f64(inp["v"]),
                                     wl.to_f64(inp["sink"]), case.window, case.theta, wl.ROT_DIMS,
                                     rows, case.hq)
     og = wl.to_f64(out[0, pos])                                       # [len(pos), Hq, 128]
     lg = wl.to_f64(lse[0][:, pos])                                    # [Hq, len(pos)]
-    o_gpu = np.stack([og[a, h] for a in range(len(pos)) for h in hs])
-    l_gpu = np.array([lg[h, a] for a in range(len(pos)) for h in hs])
+    o_gpu = np.stack([og[a, h] for a in range(len(pos)) for h in head_sets[a]])
+    l_gpu = np.array([lg[h, a] for a in range(len(pos)) for h in head_sets[a]])
     compare(o_gpu, o_ref, l_gpu, l_ref, case.name)
     assert torch.isfinite(out).all() and torch.isfinite(lse).all()
     del inp, out, lse

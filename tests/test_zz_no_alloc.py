@@ -4,9 +4,10 @@ mimo_attn_sparse_noalloc is for callers that cannot allocate device memory when
 they call attention (for example a serving loop whose KV pools already hold nearly
 all of HBM, or a plug-in whose host framework owns every allocation). It keeps its
 split-KV partials in a fixed 8 MiB array inside the library. This test calls it
-through the C ABI twice in a row, on different inputs, and checks each result
-against mimo_attn_sparse with a caller-provided workspace, so stale contents left
-in the shared array by the first call cannot leak into the second. It also checks
+through the C ABI twice in a row, on different inputs, and then a third time with a
+smaller plan, and checks each result against mimo_attn_sparse with a caller-provided
+workspace, so stale contents left in the shared array by an earlier call cannot leak
+into a later one. It also checks
 that sizes needing more scratch than the array holds are refused before any launch.
 This file sorts last so that a run stopping at the first failure has already run
 every other test; it also passes on its own in a fresh process.
@@ -51,10 +52,16 @@ def test_noalloc_matches_workspace_version_twice(cuda_device):
     recent, cap = 128, 20000
     a = _case(501, cuda_device)
     b = _case(502, cuda_device)
+    # a third call with a smaller batch and fewer selected tokens: fewer chunks per
+    # (sequence, KV head) and a different slot layout in the array than the calls before it
+    c = _case(503, cuda_device, B=2, n_sel=300)
     need = _lib.workspace_size(4, 64, 4, op=_lib.MIMO_OP_SPARSE, capacity=cap, recent=recent,
                                n_sel=1024)
+    need_c = _lib.workspace_size(2, 64, 4, op=_lib.MIMO_OP_SPARSE, capacity=cap, recent=recent,
+                                 n_sel=300)
     assert 0 < need <= 8 * 1024 * 1024, need      # the case really uses the scratch array
-    for inp in (a, b):                             # two calls in a row, different inputs
+    assert 0 < need_c < need, need_c
+    for inp in (a, b, c):                          # calls in a row, different inputs and plans
         st, out, lse = _noalloc(inp, recent, cap)
         assert st == 0, _lib.STATUS.get(st)
         ref_out, ref_lse = _lib.sparse(inp["q"], inp["k_cache"], inp["v_cache"], inp["lengths"],
