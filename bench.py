@@ -194,30 +194,27 @@ def roofline_tensor(flops_per_launch, ms_per_launch, peak, tag, traffic=None):
 
 
 # ----------------------------------------------------------------------------- CPU oracle baseline
-def oracle_swa_sample(case: wl.PrefillCase, positions: int):
-    """Times the float64 oracle, as it stands, on query positions 0..positions-1 (all
-    heads) of the SWA-layer workload; returns (TFLOP/s, description, threads, seconds)."""
-    from oracle import ref
-    from threadpoolctl import threadpool_limits
-    inp = wl.prefill_inputs(case.batch, positions, case.hq, case.hkv, seed=case.seed)
-    q = wl.to_f64(inp["q"])
-    k, v, s = wl.to_f64(inp["k"]), wl.to_f64(inp["v"]), wl.to_f64(inp["sink"])
-    with threadpool_limits(1):
-        t0 = time.perf_counter()
-        ref.prefill(q, k, v, s, case.window, case.theta, wl.ROT_DIMS)
-        dt = time.perf_counter() - t0
-    pairs = swa_pairs(positions, case.window)
-    flops = 2.0 * (wl.DQK + wl.DV) * pairs * case.hq * case.batch
-    desc = (f"float64 oracle, all {case.hq} heads of query positions 0..{positions - 1} of the "
-            f"n={case.seqlen} SWA layer (same window, RoPE and sinks), one thread")
-    return flops / dt / 1e12, desc, 1, dt
+def run_oracle_harness(*extra, timeout=900):
+    """Runs the float64 oracle's timing harness (``python -m oracle.baseline``) as a separate
+    process that never touches a GPU, on all host cores; returns its JSON object."""
+    cmd = [sys.executable, "-m", "oracle.baseline", *[str(x) for x in extra]]
+    res = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=timeout)
+    if res.returncode != 0:
+        raise RuntimeError(f"oracle harness failed: {res.stderr[-500:]}")
+    return json.loads(res.stdout.strip().splitlines()[-1])
 
 
-def oracle_positions_for(case, seconds):
-    """Query positions whose oracle run takes about ``seconds`` on this host."""
-    _, _, _, dt = oracle_swa_sample(case, 64)
-    per_pos = dt / 64
-    return int(max(32, min(4096, seconds / per_pos)))
+def cpu_baseline_line(budget=3.0):
+    """The oracle on every configuration (full where it finishes in seconds, a row sample
+    extrapolated by work otherwise); ``value`` is the headline SWA-prefill throughput."""
+    h = run_oracle_harness("--budget", budget)
+    w = h["workloads"]
+    per = {k: [v["s"], v["how"][:5]] for k, v in w.items()}
+    return {"value": w["swa_prefill"]["rate"], "unit": "TFLOP/s", "cores": h["cores"], "kind": "oracle",
+            "sample": (f"float64 oracle, {h['cores']} processes x 1 BLAS thread: SWA n=32768 random rows x heads "
+                       f"({budget:g} s per process), extrapolated by pairs; per_config = est. seconds per call "
+                       "(full|extra[polated])"),
+            "per_config": per}
 
 
 # ----------------------------------------------------------------------------- workloads
@@ -236,6 +233,40 @@ def bench_prefill(case, steps, warmup, peaks, tag, dev, stream):
     err = _lib.last_device_error()
     res = {"inp": inp, "ms_total": ms, "flops": flops, "bytes": bytes_, "device_error": err}
     return res
+
+
+def bench_tiny_prefill(steps, peaks, tag, dev, stream):
+    """Tiny SWA+sink prefill (n=1024, 8 Q / 1 KV, W=128): 5.9 MB of inputs and outputs, below
+    L2, so every launch is preceded by a 256 MB write that flushes L2 and is timed alone with
+    CUDA events on the launching stream."""
+    from hybrid_sliding_window_sink_b200 import _lib
+    case = wl.TINY_SWA_PREFILL
+    inp = wl.case_prefill_inputs(case, device=dev)
+    out = torch.empty(case.batch, case.seqlen, case.hq, wl.DV, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(case.batch, case.hq, case.seqlen, dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        _lib.prefill(inp["q"], inp["k"], inp["v"], inp["sink"], window=case.window,
+                     rope_theta=case.theta, rot_dims=wl.ROT_DIMS, out=out, lse=lse, stream=stream)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    with torch.cuda.stream(stream):
+        for e0, e1 in ev:
+            flush.fill_(1)
+            e0.record(stream)
+            step()
+            e1.record(stream)
+    torch.cuda.synchronize()
+    ms = statistics.median(e0.elapsed_time(e1) for e0, e1 in ev)
+    flops, bytes_ = prefill_work(case)
+    del inp, out, lse, flush
+    return {"ms": round(ms, 5), "tflops": round(flops / (ms * 1e-3) / 1e12, 2),
+            "frac": round(bytes_ / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+            "device_error": _lib.last_device_error()}
 
 
 def bench_chunk_prefill(steps, warmup, peaks, tag, dev, stream, chunk=16384, prefix=16384):
@@ -460,13 +491,6 @@ def fp8_decode_layer_bytes(lengths, hq, hkv, kind, cap):
     return float(kv + B * hq * wl.DQK * 2 + B * hq * wl.DV * 2 + B * hq * 4 + hq * 4 + B * 4)
 
 
-def _random_e4m3(shape, g, dev):
-    """Random E4M3 bytes (NaN patterns replaced by 0) for timing runs."""
-    b = torch.randint(0, 256, shape, generator=g, device=dev, dtype=torch.int32)
-    b = torch.where((b & 0x7F) == 0x7F, torch.zeros_like(b), b)
-    return b.to(torch.uint8)
-
-
 def bench_fp8_decode_step(steps, warmup, peaks, tag, dev, stream):
     """The hybrid decode step of bench_decode_step over FP8 caches (E4M3 K/V with
     per-(token, KV head) fp32 scales): 39 SWA rings of 128 slots, 9 GA layers on one padded
@@ -478,16 +502,16 @@ def bench_fp8_decode_step(steps, warmup, peaks, tag, dev, stream):
     g = torch.Generator(device=dev)
     g.manual_seed(cs.seed + 9)
     mk_scale = lambda *sh: torch.empty(*sh, device=dev).uniform_(0.002, 0.01, generator=g)  # noqa: E731
-    ga = (_random_e4m3((cg.batch, cg.capacity, cg.hkv, wl.DQK), g, dev),
-          _random_e4m3((cg.batch, cg.capacity, cg.hkv, wl.DV), g, dev),
+    ga = (wl.random_e4m3((cg.batch, cg.capacity, cg.hkv, wl.DQK), g, dev),
+          wl.random_e4m3((cg.batch, cg.capacity, cg.hkv, wl.DV), g, dev),
           mk_scale(cg.batch, cg.capacity, cg.hkv), mk_scale(cg.batch, cg.capacity, cg.hkv))
     layers = []
     for kind in wl.layer_pattern():
         q = torch.randn(cs.batch, cs.hq, wl.DQK, generator=g, device=dev).to(torch.bfloat16)
         sink = torch.randn(cs.hq, generator=g, device=dev)
         if kind == 1:
-            cache = (_random_e4m3((cs.batch, cs.capacity, cs.hkv, wl.DQK), g, dev),
-                     _random_e4m3((cs.batch, cs.capacity, cs.hkv, wl.DV), g, dev),
+            cache = (wl.random_e4m3((cs.batch, cs.capacity, cs.hkv, wl.DQK), g, dev),
+                     wl.random_e4m3((cs.batch, cs.capacity, cs.hkv, wl.DV), g, dev),
                      mk_scale(cs.batch, cs.capacity, cs.hkv), mk_scale(cs.batch, cs.capacity, cs.hkv))
         else:
             cache = ga
@@ -614,6 +638,83 @@ def bench_sparse(steps, warmup, peaks, tag, dev, stream, calls=16):
 
 
 # ----------------------------------------------------------------------------- main
+#: Wall-clock seconds the reference arm spends in all (warm-up + timed steps), and the number
+#: of host processes it uses (0 = every core this process may run on).
+REF_SECONDS = 120.0
+REF_CORES = 0
+
+
+def reference_arm(args, warmup, case):
+    """``--impl reference``: the float64 oracle on the host cores, on the headline workload's
+    row sample, each step a bounded sample; rank 0 only."""
+    world, rank, _ = D.env_world()
+    if rank != 0:
+        return
+    budget = max(0.02, REF_SECONDS / (args.steps + warmup))
+    h = run_oracle_harness("--only", "swa_prefill", "--steps", args.steps, "--warmup", warmup,
+                           "--budget", budget, "--cores", REF_CORES)
+    work = sum(w for w, _ in h["steps"])
+    wall = sum(t for _, t in h["steps"])
+    value = work / wall / 1e12
+    desc = (f"float64 oracle, {h['cores']} processes x 1 BLAS thread, random rows x heads of the "
+            f"n=32768 SWA layer, {budget:.2f} s per process per step")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": warmup,
+            "ms_per_step": 1e3 * wall / len(h["steps"]), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": case.name, "global_batch": case.batch, "seq_len": case.seqlen,
+                       "parallelism": "none (host CPU)"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": h["cores"],
+                             "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+
+
+def _r(x, nd=4):
+    return None if x is None else round(x, nd)
+
+
+def compact_workloads(w):
+    """The per-workload figures in short form for the JSON line (the full records go to
+    ``--detail``). ms = device time per call or step; frac = roofline fraction of the
+    measured HBM copy peak, except where bound = tensor (fraction of the bf16 GEMM peak)."""
+    out = {}
+
+    def err(name):
+        if "error" in w.get(name, {}):
+            out[name] = {"error": w[name]["error"][:120]}
+            return True
+        return name not in w
+
+    if not err("tiny_prefill"):
+        out["tiny_prefill"] = {k: w["tiny_prefill"][k] for k in ("ms", "tflops", "frac")}
+    if not err("ga_prefill"):
+        g = w["ga_prefill"]
+        out["ga_prefill"] = {"bound": "tensor", "ms": g["ms_per_step"], "tflops": g["value"],
+                             "frac": g["roofline"]["frac"], "traffic": g["roofline"]["traffic"]}
+    if not err("chunk_prefill"):
+        c = w["chunk_prefill"]
+        out["chunk_swa"] = {"ms": c["swa"]["ms"], "frac": c["swa"]["roofline"]["frac"]}
+        out["chunk_ga"] = {"bound": "tensor", "ms": c["ga"]["ms"], "tflops": c["ga"]["tflops"],
+                           "frac": c["ga"]["roofline"]["frac"]}
+    for name, short in (("hybrid_decode_step", "decode_step"), ("fp8_decode_step", "fp8_step"),
+                        ("mtp_decode_step", "mtp_step")):
+        if err(name):
+            continue
+        d = w[name]
+        out[short] = {"ms": d["ms_per_step"], "gbs": d["value"], "frac": d["roofline"]["frac"],
+                      "ga_ms": d["ms_ga_layer"], "ga_frac": d["ga_layer"]["frac"],
+                      "swa_ms": d["ms_swa_layer"], "swa_frac": d["swa_layer"]["frac"]}
+    if not err("token_select"):
+        t = w["token_select"]
+        out["select"] = {"ms": t["ms_per_call"], "gbs": t["value"], "frac": t["roofline"]["frac"]}
+    if not err("sparse_decode"):
+        t = w["sparse_decode"]
+        out["sparse"] = {"us": _r(t["ms_per_call"] * 1e3, 2), "gbs": t["value"], "frac": t["roofline"]["frac"]}
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -623,36 +724,14 @@ def main():
     ap.add_argument("--only-main", action="store_true", help="skip the extra workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--detail", default=None, help="also write the full per-workload records here")
     args = ap.parse_args()
     warmup = max(3, args.warmup)
     case = wl.SWA_PREFILL
     peaks, tag = load_peaks()
 
     if args.impl == "reference":
-        world, rank, _ = D.env_world()
-        if rank != 0:
-            return
-        # size each step so that warm-up + steps take about two minutes in all
-        positions = oracle_positions_for(case, 120.0 / (args.steps + warmup))
-        for _ in range(warmup):
-            oracle_swa_sample(case, positions)
-        times, vals = [], []
-        for _ in range(args.steps):
-            v, desc, cores, dt = oracle_swa_sample(case, positions)
-            vals.append(v)
-            times.append(dt)
-        value = sum(v * t for v, t in zip(vals, times)) / sum(times)
-        line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
-                "n_gpus": args.gpus, "steps": args.steps, "warmup": warmup,
-                "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True,
-                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": {"workload": case.name, "global_batch": case.batch, "seq_len": case.seqlen,
-                           "parallelism": "none (host CPU)"},
-                "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores,
-                                 "kind": "oracle", "sample": desc},
-                "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
-                        "d2h_bytes_per_step": 0}}
-        print(json.dumps(line))
+        reference_arm(args, warmup, case)
         return
 
     world, rank = D.init("nccl")
@@ -675,20 +754,21 @@ def main():
     del res["inp"]
     torch.cuda.empty_cache()
 
+    roof = roofline_hbm(bytes_, ms_step, peaks, tag,
+                        traffic_for("prefill_swa_kernel", case.batch * case.hkv * -(-case.seqlen // 16)))
+    roof.pop("peak_source")
+    tens = roofline_tensor(flops, ms_step, peaks["bf16_tflops"], tag)
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": warmup, "ms_per_step": round(ms_step, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic N(0,1) bf16 Q/K/V, fp32 N(0,1) sinks, seeded",
+        "data": "synthetic",
         "config": {"workload": case.name, "global_batch": case.batch * world, "seq_len": case.seqlen,
-                   "parallelism": f"dp{world} (independent problems per rank)",
-                   "l2": "inputs larger than L2 (1.52 GB per step)"},
-        "roofline": roofline_hbm(bytes_, ms_step, peaks, tag,
-                                 traffic_for("prefill_swa_kernel",
-                                             case.batch * case.hkv * -(-case.seqlen // 16))),
-        "tensor": roofline_tensor(flops, ms_step, peaks["bf16_tflops"], tag),
+                   "parallelism": f"dp{world}", "l2": "inputs > L2"},
+        "roofline": roof, "peaks": tag,
+        "tensor": {"achieved": tens["achieved"], "frac": tens["frac"]},
         "gpu_launches": args.steps,
-        "clocks": clk,
+        "clocks": {k: clk.get(k) for k in ("sm_mhz", "sm_max_mhz", "reasons")},
         "device_error": res["device_error"],
     }
 
@@ -702,65 +782,49 @@ def main():
         torch.cuda.empty_cache()
 
     # ---- the other workloads (single GPU figures, rank 0 reports its own)
+    wls = {}
     if not args.only_main:
-        wls = {}
         ksteps = max(3, min(args.steps // 20, 10))
-        try:
+
+        def attempt(name, fn):
+            try:
+                wls[name] = fn()
+            except Exception as e:  # report, do not hide
+                wls[name] = {"error": repr(e)}
+            torch.cuda.empty_cache()
+
+        attempt("tiny_prefill", lambda: bench_tiny_prefill(max(20, ksteps), peaks, tag, dev, stream))
+
+        def ga_prefill():
             ga = bench_prefill(wl.GA_PREFILL, ksteps, 3, peaks, tag, dev, stream)
             ms_ga = ga["ms_total"] / ksteps
-            wls["ga_prefill"] = {
-                "workload": wl.GA_PREFILL.name, "value": round(ga["flops"] / (ms_ga * 1e-3) / 1e12, 2),
-                "unit": "TFLOP/s", "ms_per_step": round(ms_ga, 4),
-                "roofline": roofline_tensor(ga["flops"], ms_ga, peaks["bf16_tflops"], tag,
-                                            traffic_for("prefill_ga_kernel", wl.GA_PREFILL.seqlen)),
-                "device_error": ga["device_error"]}
-            del ga
-            torch.cuda.empty_cache()
-        except Exception as e:  # report, do not hide
-            wls["ga_prefill"] = {"error": repr(e)}
-        try:
-            wls["chunk_prefill"] = bench_chunk_prefill(max(3, ksteps), 3, peaks, tag, dev, stream)
-        except Exception as e:
-            wls["chunk_prefill"] = {"error": repr(e)}
-        try:
-            wls["hybrid_decode_step"] = bench_decode_step(max(3, ksteps), 3, peaks, tag, dev, stream)
-            wls["hybrid_decode_step"]["workload"] = "hybrid decode step, 48 layers, B=64"
-            torch.cuda.empty_cache()
-        except Exception as e:
-            wls["hybrid_decode_step"] = {"error": repr(e)}
-        try:
-            wls["fp8_decode_step"] = bench_fp8_decode_step(max(3, ksteps), 3, peaks, tag, dev, stream)
-            wls["fp8_decode_step"]["workload"] = "hybrid decode step over FP8 caches, 48 layers, B=64"
-            torch.cuda.empty_cache()
-        except Exception as e:
-            wls["fp8_decode_step"] = {"error": repr(e)}
-        try:
-            wls["mtp_decode_step"] = bench_mtp_step(max(3, ksteps), 3, peaks, tag, dev, stream)
-            wls["mtp_decode_step"]["workload"] = "MTP verification step (1+3 tokens), 48 layers, B=64"
-            torch.cuda.empty_cache()
-        except Exception as e:
-            wls["mtp_decode_step"] = {"error": repr(e)}
-        try:
-            wls["token_select"] = bench_select(max(3, ksteps), 3, peaks, tag, dev, stream)
-            torch.cuda.empty_cache()
-        except Exception as e:
-            wls["token_select"] = {"error": repr(e)}
-        try:
-            wls["sparse_decode"] = bench_sparse(max(5, ksteps), 3, peaks, tag, dev, stream)
-            wls["sparse_decode"]["workload"] = wl.SPARSE_DECODE.name
-            torch.cuda.empty_cache()
-        except Exception as e:
-            wls["sparse_decode"] = {"error": repr(e)}
-        line["workloads"] = wls
+            return {"workload": wl.GA_PREFILL.name, "value": round(ga["flops"] / (ms_ga * 1e-3) / 1e12, 2),
+                    "unit": "TFLOP/s", "ms_per_step": round(ms_ga, 4),
+                    "roofline": roofline_tensor(ga["flops"], ms_ga, peaks["bf16_tflops"], tag,
+                                                traffic_for("prefill_ga_kernel", wl.GA_PREFILL.seqlen)),
+                    "device_error": ga["device_error"]}
 
-    # ---- CPU oracle baseline (rank 0, N = 1 only)
+        attempt("ga_prefill", ga_prefill)
+        attempt("chunk_prefill", lambda: bench_chunk_prefill(max(3, ksteps), 3, peaks, tag, dev, stream))
+        attempt("hybrid_decode_step", lambda: bench_decode_step(max(3, ksteps), 3, peaks, tag, dev, stream))
+        attempt("fp8_decode_step", lambda: bench_fp8_decode_step(max(3, ksteps), 3, peaks, tag, dev, stream))
+        attempt("mtp_decode_step", lambda: bench_mtp_step(max(3, ksteps), 3, peaks, tag, dev, stream))
+        attempt("token_select", lambda: bench_select(max(3, ksteps), 3, peaks, tag, dev, stream))
+        attempt("sparse_decode", lambda: bench_sparse(max(5, ksteps), 3, peaks, tag, dev, stream))
+        line["workloads"] = compact_workloads(wls)
+
+    # ---- CPU oracle baseline (rank 0, N = 1 only), in a process of its own on the host cores
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, desc, cores, dt = oracle_swa_sample(case, oracle_positions_for(case, 15.0))
-        line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                                "sample": desc, "seconds": round(dt, 2)}
+        try:
+            line["cpu_baseline"] = cpu_baseline_line()
+        except Exception as e:
+            line["cpu_baseline"] = {"error": repr(e)[:200]}
 
     if rank == 0:
-        print(json.dumps(line))
+        if args.detail:
+            with open(args.detail, "w") as f:
+                json.dump({"line": line, "workloads": wls, "clocks": clk}, f, indent=1, default=str)
+        print(json.dumps(line, separators=(",", ":")))
     D.finalize()
 
 

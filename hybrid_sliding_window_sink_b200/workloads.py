@@ -184,9 +184,8 @@ def integer_qk(batch, hq, hkv, capacity, *, seed, device="cpu", lo=-2, hi=2):
 def random_e4m3(shape, g, device):
     """Uniformly random E4M3 bytes with the two NaN patterns replaced by 0 (a cache holds
     no NaN), drawn with generator ``g`` on ``device``."""
-    b = torch.randint(0, 256, shape, generator=g, device=device, dtype=torch.int32)
-    b = torch.where((b & 0x7F) == 0x7F, torch.zeros_like(b), b)
-    return b.to(torch.uint8)
+    b = torch.randint(0, 256, shape, generator=g, device=device, dtype=torch.uint8)
+    return b.masked_fill_((b & 0x7F) == 0x7F, 0)
 
 
 def random_fp8_cache(batch, capacity, hkv, *, seed, device="cpu", scale_lo=0.002, scale_hi=0.01):

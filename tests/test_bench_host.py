@@ -85,7 +85,8 @@ def test_recorded_traffic_files_exist():
 
 
 def _run_reference(monkeypatch, capsys, rank="0"):
-    monkeypatch.setattr(bench, "oracle_positions_for", lambda case, seconds: 32)
+    monkeypatch.setattr(bench, "REF_SECONDS", 0.5)
+    monkeypatch.setattr(bench, "REF_CORES", 2)
     monkeypatch.setattr("sys.argv", ["bench.py", "--impl", "reference", "--steps", "2", "--warmup", "3"])
     monkeypatch.setenv("RANK", rank)
     monkeypatch.setenv("WORLD_SIZE", "2" if rank != "0" else "1")
@@ -95,8 +96,8 @@ def _run_reference(monkeypatch, capsys, rank="0"):
 
 
 def test_reference_arm_json_contract(monkeypatch, capsys):
-    """`bench.py --impl reference` (the float64 oracle on host cores, on a 32-position sample
-    here): one JSON line with the contract's keys, the oracle as its cpu_baseline."""
+    """`bench.py --impl reference` (the float64 oracle on host cores, two processes and a
+    short budget here): one JSON line with the contract's keys, the oracle as its cpu_baseline."""
     lines = _run_reference(monkeypatch, capsys)
     assert len(lines) == 1
     d = json.loads(lines[0])
@@ -114,3 +115,48 @@ def test_reference_arm_json_contract(monkeypatch, capsys):
 
 def test_reference_arm_other_ranks_print_nothing(monkeypatch, capsys):
     assert _run_reference(monkeypatch, capsys, rank="1") == []
+
+
+def _fake_workloads():
+    hb = lambda f: {"bound": "hbm", "achieved": 4321.5, "peak": 6452.2, "unit": "GB/s", "frac": f,  # noqa: E731
+                    "traffic": 123456789012, "peak_source": "measured"}
+    step = {"value": 5123.4, "unit": "GB/s", "ms_per_step": 20.1234, "ga_layer": hb(0.8123),
+            "swa_layer": hb(0.6123), "roofline": hb(0.7912), "ms_ga_layer": 2.1234, "ms_swa_layer": 0.01234}
+    return {
+        "tiny_prefill": {"ms": 0.01234, "tflops": 51.23, "frac": 0.0712, "device_error": 0},
+        "ga_prefill": {"value": 1012.34, "ms_per_step": 21.7234, "device_error": 0,
+                       "roofline": {"frac": 0.6123, "traffic": 1434567890}},
+        "chunk_prefill": {"swa": {"ms": 0.2123, "roofline": hb(0.5123)},
+                          "ga": {"ms": 16.1234, "tflops": 1012.34, "roofline": {"frac": 0.6123}}},
+        "hybrid_decode_step": dict(step), "fp8_decode_step": dict(step), "mtp_decode_step": dict(step),
+        "token_select": {"ms_per_call": 0.5812, "value": 5766.1, "roofline": hb(0.8812)},
+        "sparse_decode": {"ms_per_call": 0.00812, "value": 2961.2, "roofline": hb(0.4512)},
+    }
+
+
+def test_bench_line_fits_the_driver_tail():
+    """The whole JSON line, with every workload and the CPU baseline, stays well under the
+    ~3000 characters of stdout the driver keeps, so every figure is recorded."""
+    w = bench.compact_workloads(_fake_workloads())
+    assert set(w) == {"tiny_prefill", "ga_prefill", "chunk_swa", "chunk_ga", "decode_step", "fp8_step",
+                      "mtp_step", "select", "sparse"}
+    line = {"metric": bench.METRIC, "value": 376.155, "unit": "TFLOP/s", "n_gpus": 1, "steps": 20,
+            "warmup": 5, "ms_per_step": 0.45584, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.SWA_PREFILL.name, "global_batch": 1, "seq_len": 32768,
+                       "parallelism": "dp1", "l2": "inputs > L2"},
+            "roofline": {"bound": "hbm", "achieved": 3330.9, "peak": 6452.2, "unit": "GB/s", "frac": 0.5079,
+                         "traffic": 1419895808}, "peaks": "measured",
+            "tensor": {"achieved": 376.15, "frac": 0.2261}, "gpu_launches": 20,
+            "clocks": {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]},
+            "device_error": 0,
+            "e2e": {"value": 6.225, "unit": "TFLOP/s", "h2d_bytes_per_step": 973078784,
+                    "d2h_bytes_per_step": 545259520, "ms_per_step": 27.545},
+            "workloads": w,
+            "cpu_baseline": {"value": 0.0123456789, "unit": "TFLOP/s", "cores": 224, "kind": "oracle",
+                             "sample": "x" * 200,
+                             "per_config": {k: [12345.67, "extra"] for k in
+                                            ("tiny_prefill", "swa_prefill", "ga_prefill", "swa_decode",
+                                             "ga_decode", "sparse_decode")}}}
+    text = json.dumps(line, separators=(",", ":"))
+    assert len(text) < 2600, len(text)
