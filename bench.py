@@ -23,7 +23,6 @@ import os
 import statistics
 import subprocess
 import sys
-import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -50,54 +49,52 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons while the timed loop runs."""
+    """SM clock and clock-event (throttle) reasons sampled through NVML every millisecond by a
+    thread while the timed loop runs (the headline's timed region is only milliseconds long,
+    too short for nvidia-smi's sampling interval). Read-only queries."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock-event reason bits
+    REASONS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+               "hw_thermal_slowdown": 0x40}
 
-    def __init__(self, device_index: int):
-        self.proc = None
-        self.path = None
+    def __init__(self, device_index: int, period_s: float = 0.001):
+        import threading
+        self.samples, self.reasons, self.smax, self.err = [], set(), None, None
+        self._stop = threading.Event()
         try:
+            import pynvml
+            pynvml.nvmlInit()
             uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
-            fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
-            os.close(fd)
-            self.out = open(self.path, "w")
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", uuid, f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "20"],
-                stdout=self.out, stderr=subprocess.DEVNULL)
-        except Exception:
-            self.proc = None
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.smax = float(pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM))
+        except Exception as e:  # no NVML: report it in the line
+            self.err = repr(e)[:80]
+            return
+        self._thread = threading.Thread(target=self._run, args=(period_s,), daemon=True)
+        self._thread.start()
+
+    def _run(self, period_s):
+        nv, h = self._nv, self._h
+        while not self._stop.is_set():
+            try:
+                self.samples.append(float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)))
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                for name, bit in self.REASONS.items():
+                    if bits & bit:
+                        self.reasons.add(name)
+            except Exception as e:
+                self.err = repr(e)[:80]
+                return
+            time.sleep(period_s)
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.out.close()
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        with open(self.path) as f:
-            for line in f:
-                parts = [x.strip() for x in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    sm.append(float(parts[1]))
-                    smax = float(parts[2])
-                except ValueError:
-                    continue
-                for nm, val in zip(names, parts[5:9]):
-                    if val.lower().startswith("active"):
-                        reasons.add(nm)
-        os.unlink(self.path)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "samples": len(sm), "reasons": sorted(reasons)}
+        if self.err is not None and not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [f"NVML unavailable: {self.err}"]}
+        self._stop.set()
+        self._thread.join(timeout=2)
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.smax,
+                "samples": len(self.samples), "reasons": sorted(self.reasons)}
 
 
 # ----------------------------------------------------------------------------- measured traffic
@@ -148,11 +145,12 @@ class DeviceError(RuntimeError):
     pass
 
 
-def timed(fn, steps, warmup, stream, flush=None):
+def timed(fn, steps, warmup, stream, flush=None, clocks=None):
     """Run ``warmup`` untimed steps, then time exactly ``steps`` with CUDA events on
     ``stream``, bracketed by barrier + synchronize. Returns elapsed ms of this rank.
     Raises DeviceError (before timing) if a warm-up step set the library's device error
-    word, so that a broken kernel is not timed."""
+    word, so that a broken kernel is not timed. ``clocks``: a list that receives a
+    ClockSampler's record of the timed region."""
     from hybrid_sliding_window_sink_b200 import _lib
     for _ in range(warmup):
         fn()
@@ -162,6 +160,7 @@ def timed(fn, steps, warmup, stream, flush=None):
         raise DeviceError(f"device error word {err} set during warm-up")
     D.barrier()
     torch.cuda.synchronize()
+    sampler = ClockSampler(torch.cuda.current_device()) if clocks is not None else None
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
@@ -171,6 +170,8 @@ def timed(fn, steps, warmup, stream, flush=None):
         fn()
     e1.record(stream)
     torch.cuda.synchronize()
+    if sampler is not None:
+        clocks.append(sampler.stop())
     D.barrier()
     return e0.elapsed_time(e1)
 
@@ -218,7 +219,7 @@ def cpu_baseline_line(budget=3.0):
 
 
 # ----------------------------------------------------------------------------- workloads
-def bench_prefill(case, steps, warmup, peaks, tag, dev, stream):
+def bench_prefill(case, steps, warmup, peaks, tag, dev, stream, clocks=None):
     from hybrid_sliding_window_sink_b200 import _lib
     inp = wl.case_prefill_inputs(case, device=dev)
     out = torch.empty(case.batch, case.seqlen, case.hq, wl.DV, dtype=torch.bfloat16, device=dev)
@@ -228,7 +229,7 @@ def bench_prefill(case, steps, warmup, peaks, tag, dev, stream):
         _lib.prefill(inp["q"], inp["k"], inp["v"], inp["sink"], window=case.window,
                      rope_theta=case.theta, rot_dims=wl.ROT_DIMS, out=out, lse=lse, stream=stream)
 
-    ms = timed(step, steps, warmup, stream)
+    ms = timed(step, steps, warmup, stream, clocks=clocks)
     flops, bytes_ = prefill_work(case)
     err = _lib.last_device_error()
     res = {"inp": inp, "ms_total": ms, "flops": flops, "bytes": bytes_, "device_error": err}
@@ -340,34 +341,39 @@ def e2e_prefill(case, steps, dev, stream):
     return ms / steps, h2d, d2h
 
 
-def bench_decode_step(steps, warmup, peaks, tag, dev, stream):
+def bench_decode_step(steps, warmup, peaks, tag, dev, stream, batch_range=None):
     """One decode step over the 48-layer hybrid pattern (B=64): 39 SWA ring layers with
-    distinct caches and 9 GA layers reading one padded linear cache (131072 slots)."""
+    distinct caches and 9 GA layers reading one padded linear cache (131072 slots). With
+    ``batch_range`` = (lo, hi) only sequences [lo, hi) of the batch (their lengths, caches,
+    queries and outputs): this rank's share when the step is partitioned across ranks."""
     from hybrid_sliding_window_sink_b200 import _lib
     cs, cg = wl.HYBRID_DECODE_SWA, wl.HYBRID_DECODE_GA
     L = wl.lengths_uniform(cs.batch, cs.min_len, cs.max_len, seed=cs.seed)
+    lo, hi = batch_range if batch_range is not None else (0, cs.batch)
+    L = L[lo:hi]
+    B = hi - lo
     Ld = L.to(dev)
     g = torch.Generator(device=dev)
-    g.manual_seed(cs.seed)
+    g.manual_seed(cs.seed + 1000 * lo)
     pattern = wl.layer_pattern()
     layers = []
-    ga_k = torch.randn(cg.batch, cg.capacity, cg.hkv, wl.DQK, generator=g, device=dev,
+    ga_k = torch.randn(B, cg.capacity, cg.hkv, wl.DQK, generator=g, device=dev,
                        dtype=torch.float32).to(torch.bfloat16)
-    ga_v = torch.randn(cg.batch, cg.capacity, cg.hkv, wl.DV, generator=g, device=dev,
+    ga_v = torch.randn(B, cg.capacity, cg.hkv, wl.DV, generator=g, device=dev,
                        dtype=torch.float32).to(torch.bfloat16)
     for li, kind in enumerate(pattern):
         hkv = cs.hkv if kind == 1 else cg.hkv
-        q = torch.randn(cs.batch, cs.hq, wl.DQK, generator=g, device=dev).to(torch.bfloat16)
+        q = torch.randn(B, cs.hq, wl.DQK, generator=g, device=dev).to(torch.bfloat16)
         sink = torch.randn(cs.hq, generator=g, device=dev)
         if kind == 1:
-            kc = torch.randn(cs.batch, cs.capacity, hkv, wl.DQK, generator=g, device=dev).to(torch.bfloat16)
-            vc = torch.randn(cs.batch, cs.capacity, hkv, wl.DV, generator=g, device=dev).to(torch.bfloat16)
+            kc = torch.randn(B, cs.capacity, hkv, wl.DQK, generator=g, device=dev).to(torch.bfloat16)
+            vc = torch.randn(B, cs.capacity, hkv, wl.DV, generator=g, device=dev).to(torch.bfloat16)
         else:
             kc, vc = ga_k, ga_v
-        out = torch.empty(cs.batch, cs.hq, wl.DV, dtype=torch.bfloat16, device=dev)
-        lse = torch.empty(cs.batch, cs.hq, dtype=torch.float32, device=dev)
+        out = torch.empty(B, cs.hq, wl.DV, dtype=torch.bfloat16, device=dev)
+        lse = torch.empty(B, cs.hq, dtype=torch.float32, device=dev)
         layers.append((kind, q, kc, vc, sink, out, lse))
-    nws = _lib.workspace_size(cg.batch, cg.hq, cg.hkv, op=_lib.MIMO_OP_DECODE,
+    nws = _lib.workspace_size(B, cg.hq, cg.hkv, op=_lib.MIMO_OP_DECODE,
                               kind=_lib.MIMO_CACHE_LINEAR, capacity=cg.capacity)
     ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
 
@@ -671,6 +677,31 @@ def reference_arm(args, warmup, case):
     print(json.dumps(line))
 
 
+def decode_shard_arm(args, warmup, peaks, tag):
+    """``--decode-shard``: the hybrid decode step (B=64, 48 layers) partitioned across the
+    ranks by sequence, each rank running its contiguous share of the batch on its GPU (no
+    exchange: sequences share nothing). value = the algorithmic bytes of all ranks over the
+    slowest rank's time (strong scaling: the total work is fixed)."""
+    world, rank = D.init("nccl")
+    _, _, local = D.env_world()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    lo, hi = D.shard_range(wl.HYBRID_DECODE_SWA.batch, rank, world)
+    res = bench_decode_step(args.steps, warmup, peaks, tag, dev, stream, batch_range=(lo, hi))
+    ms = D.max_over_ranks(res["ms_per_step"], device=dev)
+    total = D.sum_over_ranks(res["bytes_per_step"], device=dev)
+    if rank == 0:
+        print(json.dumps({"metric": "hybrid decode step HBM GB/s, sequences partitioned across ranks",
+                          "value": round(total / (ms * 1e-3) / 1e9, 1), "unit": "GB/s", "n_gpus": world,
+                          "steps": args.steps, "warmup": warmup, "ms_per_step": ms, "higher_is_better": True,
+                          "scaling": "strong", "dtype": "bf16", "data": "synthetic",
+                          "config": {"workload": "hybrid decode step, 48 layers, B=64 split by sequence",
+                                     "sequences_per_rank": [D.shard_range(64, r, world) for r in range(world)]},
+                          "roofline": roofline_hbm(total / world, ms, peaks, tag)}, separators=(",", ":")))
+    D.finalize()
+
+
 def _r(x, nd=4):
     return None if x is None else round(x, nd)
 
@@ -725,6 +756,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--detail", default=None, help="also write the full per-workload records here")
+    ap.add_argument("--decode-shard", action="store_true",
+                    help="time only the 48-layer decode step, its 64 sequences partitioned across ranks")
     args = ap.parse_args()
     warmup = max(3, args.warmup)
     case = wl.SWA_PREFILL
@@ -732,6 +765,9 @@ def main():
 
     if args.impl == "reference":
         reference_arm(args, warmup, case)
+        return
+    if args.decode_shard:
+        decode_shard_arm(args, warmup, peaks, tag)
         return
 
     world, rank = D.init("nccl")
@@ -743,9 +779,9 @@ def main():
     stream = torch.cuda.current_stream(dev)
 
     # ---- headline: SWA-layer prefill (each rank its own copy: weak scaling)
-    clocks = ClockSampler(local)
-    res = bench_prefill(case, args.steps, warmup, peaks, tag, dev, stream)
-    clk = clocks.stop()
+    clk_rec = []
+    res = bench_prefill(case, args.steps, warmup, peaks, tag, dev, stream, clocks=clk_rec)
+    clk = clk_rec[0]
     ms_rank = res["ms_total"]
     ms_max = D.max_over_ranks(ms_rank, device=dev)
     ms_step = ms_max / args.steps

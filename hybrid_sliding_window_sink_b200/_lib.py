@@ -29,8 +29,8 @@ EXPORTS = ("mimo_attn_prefill", "mimo_attn_decode", "mimo_attn_sparse", "mimo_at
            "mimo_attn_decode_mq", "mimo_attn_decode_mq_workspace_size", "mimo_attn_workspace_size",
            "mimo_attn_decode_fp8", "mimo_attn_sparse_fp8", "mimo_attn_prefill_chunk",
            "mimo_attn_cache_append", "mimo_attn_select_tokens", "mimo_attn_select_workspace_size",
-           "mimo_attn_check_indices", "mimo_attn_last_device_error", "mimo_status_string",
-           "mimo_attn_version")
+           "mimo_attn_check_indices", "mimo_attn_last_device_error", "mimo_attn_device_status",
+           "mimo_status_string", "mimo_attn_version")
 
 
 class MimoError(RuntimeError):
@@ -54,12 +54,18 @@ _LIB = None
 def lib():
     """Load libmimo_attn.so once; raise if it has not been built."""
     global _LIB
-    if _LIB is not None:
-        return _LIB
-    if not os.path.exists(LIB_PATH):
-        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+    if _LIB is None:
+        _LIB = load(LIB_PATH)
+    return _LIB
+
+
+def load(path):
+    """Load one build of the library (the product build, or a test build such as the one
+    with a short wait limit) and declare the argument types of every entry point."""
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with "
                            "`python -m hybrid_sliding_window_sink_b200.build`")
-    L = ctypes.CDLL(LIB_PATH)
+    L = ctypes.CDLL(path)
     P, I, F, LL, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_longlong, ctypes.c_size_t
     SP = ctypes.POINTER(MimoShape)
     L.mimo_attn_prefill.argtypes = [SP, P, P, P, P, I, F, I, P, P, P]
@@ -81,6 +87,8 @@ def lib():
     L.mimo_attn_check_indices.argtypes = [SP, P, P, I, I, I, P, P]
     L.mimo_attn_last_device_error.argtypes = []
     L.mimo_attn_last_device_error.restype = ctypes.c_uint
+    L.mimo_attn_device_status.argtypes = [P]
+    L.mimo_attn_device_status.restype = I
     L.mimo_status_string.argtypes = [I]
     L.mimo_status_string.restype = ctypes.c_char_p
     L.mimo_attn_version.argtypes = []
@@ -88,7 +96,6 @@ def lib():
     for fn in ("mimo_attn_prefill", "mimo_attn_decode", "mimo_attn_sparse", "mimo_attn_sparse_noalloc",
                "mimo_attn_check_indices"):
         getattr(L, fn).restype = I
-    _LIB = L
     return L
 
 

@@ -69,13 +69,18 @@ struct DecodeParams {
   const float* k_scale;       // [B, seq_stride, Hkv] fp32 (FP8 only)
   const float* v_scale;
   int B, Hq, Hkv, group, cap, mode, chunk, nchunks, recent, n_sel, direct;
+  int nstages;                // stages in flight per CTA (decode_warp_kernel)
   float scale_log2;           // softmax scale * log2(e)
   unsigned* err;
 };
 
-// Number of keys of unit (b, .) and the size of the recent part (sparse).
+// Number of keys of unit (b, .) and the size of the recent part (sparse). Lengths outside
+// [0, capacity] (linear and sparse) are clamped; debug builds also record them.
 __device__ __forceinline__ int dec_unit_keys(const DecodeParams& p, int b, int& nw, int& L) {
   L = p.lengths[b];
+#ifdef MIMO_DEBUG
+  if (L < 0 || (p.mode != kModeRing && L > p.cap)) atomicOr(p.err, kErrBadLength);
+#endif
   L = L < 0 ? 0 : L;
   if (p.mode == kModeRing) {
     nw = 0;
@@ -97,6 +102,12 @@ __device__ __forceinline__ int dec_token(const DecodeParams& p, int b, int g, in
   if (p.mode != kModeSparse) return t;
   if (t < nw) return L - nw + t;
   const int x = __ldg(p.sel + (static_cast<long long>(b) * p.Hkv + g) * p.n_sel + (t - nw));
+#ifdef MIMO_DEBUG
+  // a real entry must lie outside the recent window and above its predecessor
+  if (x < -1 || x >= L - nw || (x >= 0 && t > nw && __ldg(p.sel + (static_cast<long long>(b) * p.Hkv + g) * p.n_sel +
+                                                          (t - nw - 1)) >= x))
+    atomicOr(p.err, kErrBadIndex);
+#endif
   if (x < 0) return -1;
   return x < p.cap - 1 ? x : p.cap - 1;
 }

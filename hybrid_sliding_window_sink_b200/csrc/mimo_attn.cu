@@ -15,6 +15,7 @@
 #include "ptx.cuh"
 #include "decode.cuh"
 #include "decode_mq.cuh"
+#include "decode_warp.cuh"
 #include "select.cuh"
 #include "prefill.cuh"
 #include "prefill_swa.cuh"
@@ -22,7 +23,29 @@
 
 namespace mimo {
 __device__ unsigned g_device_error = 0;
+
+#ifdef MIMO_TEST_HOOKS
+// Test builds only: one warp waits on an mbarrier that nothing ever arrives on, through the
+// same bounded wait every kernel uses; the wait must give up and set the error word.
+__global__ void stuck_wait_kernel(unsigned* err) {
+  __shared__ __align__(8) unsigned long long bar;
+  __shared__ int abort_flag;
+  const uint32_t b = smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    mbar_init(b, 1);
+    abort_flag = 0;
+    mbar_fence_init();
+  }
+  __syncwarp();
+  const bool ok = mbar_wait(b, 0, &abort_flag, err);
+  if (threadIdx.x == 0 && ok) atomicOr(err, 0x80000000u);   // would mean the wait "completed"
 }
+#endif
+}
+
+#ifdef MIMO_TEST_HOOKS
+extern "C" int mimo_attn_test_stuck_wait(void* stream);
+#endif
 
 #ifdef MIMO_TRACE
 // Debug builds only: device buffer that receives per-phase timestamps of the prefill kernels.
@@ -321,6 +344,53 @@ DecodePlan plan_decode(const mimo_shape* s, int mode, int cap, int recent, int n
   return pl;
 }
 
+// Plan of the bf16 decode calls. Units of at most 256 keys (the SWA ring) and sparse key lists
+// run on decode_warp_kernel (one warp per CTA): a ring unit is one chunk finalised in place,
+// with two stages of 32 keys in flight; a sparse unit is cut into chunks of 64 keys (both
+// stages in flight at once) merged by the combine. Longer units (GA linear caches) use the
+// four-warp decode_split_kernel plan (*stages = 0).
+DecodePlan plan_decode_warp(const mimo_shape* s, int mode, int cap, int recent, int n_sel, int sms,
+                            int* stages) {
+  long long total = mode == mimo::kModeSparse ? static_cast<long long>(recent) + n_sel : cap;
+  if (total < 1) total = 1;
+  if (mode != mimo::kModeSparse && total > 256) {
+    *stages = 0;
+    return plan_decode(s, mode, cap, recent, n_sel, sms);
+  }
+  DecodePlan pl{};
+  *stages = 2;
+  pl.chunk = mode == mimo::kModeSparse ? 64 : static_cast<int>((total + 31) / 32 * 32);
+  if (pl.chunk > total) pl.chunk = static_cast<int>((total + 31) / 32 * 32);
+  pl.nchunks = static_cast<int>((total + pl.chunk - 1) / pl.chunk);
+  pl.direct = pl.nchunks == 1;
+  if (pl.direct) {
+    pl.bytes = 0;
+  } else {
+    const size_t rows = static_cast<size_t>(s->batch) * s->n_q_heads * pl.nchunks;
+    const size_t ml = (rows * 2 * sizeof(float) + 255) / 256 * 256;
+    pl.bytes = ml + rows * mimo::kDV * sizeof(float);
+  }
+  return pl;
+}
+
+template <int G>
+mimo_status launch_decode_warp_g(DecodeParams prm, cudaStream_t st) {
+  auto kern = mimo::decode_warp_kernel<G, 2>;
+  const int smem = mimo::dw_smem_bytes(2);
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
+    cudaGetLastError();
+    return MIMO_ERR_CUDA;
+  }
+  dim3 grid(prm.nchunks, prm.Hkv, prm.B);
+  kern<<<grid, 32, smem, st>>>(prm);
+  if (cudaGetLastError() != cudaSuccess) return MIMO_ERR_CUDA;
+  if (!prm.direct) {
+    mimo::decode_combine_kernel<<<prm.B * prm.Hq, mimo::kDV, 0, st>>>(prm);
+    if (cudaGetLastError() != cudaSuccess) return MIMO_ERR_CUDA;
+  }
+  return MIMO_OK;
+}
+
 template <int G, bool FP8 = false>
 mimo_status launch_decode_g(DecodeParams prm, cudaStream_t st) {
   auto kern = mimo::decode_split_kernel<G, FP8>;
@@ -360,7 +430,9 @@ mimo_status run_decode(const mimo_shape* s, int mode, const void* q, const void*
   const int dev = current_device();
   if (dev < 0) return MIMO_ERR_CUDA;
   const int sms = sm_count_for(dev);
-  const DecodePlan pl = plan_decode(s, mode, cap, recent, n_sel, sms);
+  int stages = 2;
+  const DecodePlan pl = fp8 ? plan_decode(s, mode, cap, recent, n_sel, sms)
+                            : plan_decode_warp(s, mode, cap, recent, n_sel, sms, &stages);
   if (pl.bytes > 0 && (!ws || ws_bytes < pl.bytes)) return MIMO_ERR_WORKSPACE;
   if (ws && !aligned(ws, 16)) return MIMO_ERR_ALIGN;
   DecodeParams prm{};
@@ -397,11 +469,21 @@ mimo_status run_decode(const mimo_shape* s, int mode, const void* q, const void*
   prm.recent = recent;
   prm.n_sel = n_sel;
   prm.direct = pl.direct;
+  prm.nstages = stages;
   prm.scale_log2 = scale_log2_of(s);
   prm.err = device_error_ptr(dev);
   if (!prm.err) return MIMO_ERR_CUDA;
   if (s->n_kv_heads > 65535) return MIMO_ERR_UNSUPPORTED;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (!fp8 && stages > 0) {
+    switch (prm.group) {
+      case 1: return launch_decode_warp_g<1>(prm, st);
+      case 2: return launch_decode_warp_g<2>(prm, st);
+      case 4: return launch_decode_warp_g<4>(prm, st);
+      case 8: return launch_decode_warp_g<8>(prm, st);
+      default: return launch_decode_warp_g<16>(prm, st);
+    }
+  }
   if (fp8) {
     switch (prm.group) {
       case 1: return launch_decode_g<1, true>(prm, st);
@@ -801,7 +883,11 @@ size_t mimo_attn_workspace_size(const mimo_shape* s, int op, int cache_kind, int
   } else {
     return 0;
   }
-  return plan_decode(s, mode, cache_capacity, recent, n_sel, sm_count_for(current_device())).bytes;
+  // one size serves both the bf16 calls (one-warp kernel plan) and the FP8 calls
+  const int sms = sm_count_for(current_device());
+  int stages = 2;
+  return std::max(plan_decode_warp(s, mode, cache_capacity, recent, n_sel, sms, &stages).bytes,
+                  plan_decode(s, mode, cache_capacity, recent, n_sel, sms).bytes);
 }
 
 mimo_status mimo_attn_check_indices(const mimo_shape* s, const int* lengths, const int* sel_idx,
@@ -832,6 +918,13 @@ unsigned int mimo_attn_last_device_error(void) {
   return v;
 }
 
+mimo_status mimo_attn_device_status(unsigned int* word) {
+  const unsigned v = mimo_attn_last_device_error();
+  if (word) *word = v;
+  if (v == 0xFFFFFFFFu) return MIMO_ERR_CUDA;
+  return v ? MIMO_ERR_DEVICE : MIMO_OK;
+}
+
 const char* mimo_status_string(mimo_status st) {
   switch (st) {
     case MIMO_OK: return "ok";
@@ -841,12 +934,22 @@ const char* mimo_status_string(mimo_status st) {
     case MIMO_ERR_ALIGN: return "misaligned data pointer";
     case MIMO_ERR_WORKSPACE: return "workspace missing or too small";
     case MIMO_ERR_CUDA: return "CUDA error";
-    case MIMO_ERR_DEVICE: return "kernel reported an internal timeout";
+    case MIMO_ERR_DEVICE: return "a kernel reported an error in the device error word";
   }
   return "unknown status";
 }
 
 int mimo_attn_version(void) { return 100; }
+
+#ifdef MIMO_TEST_HOOKS
+int mimo_attn_test_stuck_wait(void* stream) {
+  const int dev = current_device();
+  unsigned* err = dev < 0 ? nullptr : device_error_ptr(dev);
+  if (!err) return MIMO_ERR_CUDA;
+  mimo::stuck_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(err);
+  return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ERR_CUDA;
+}
+#endif
 
 }  // extern "C"
 
@@ -876,8 +979,9 @@ extern "C" mimo_status mimo_attn_sparse_noalloc(const mimo_shape* s, const void*
   if (cache_capacity < 1 || recent < 0 || n_sel < 0) return MIMO_ERR_SHAPE;
   const int dev = current_device();
   if (dev < 0) return MIMO_ERR_CUDA;
+  int stages = 2;
   const size_t need =
-      plan_decode(s, mimo::kModeSparse, cache_capacity, recent, n_sel, sm_count_for(dev)).bytes;
+      plan_decode_warp(s, mimo::kModeSparse, cache_capacity, recent, n_sel, sm_count_for(dev), &stages).bytes;
   if (need > MIMO_SPARSE_NOALLOC_SCRATCH_BYTES) return MIMO_ERR_WORKSPACE;
   void* ws = nullptr;
   size_t ws_bytes = 0;

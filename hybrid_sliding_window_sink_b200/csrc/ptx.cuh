@@ -17,10 +17,19 @@ namespace mimo {
 enum : unsigned {
   kErrWaitTimeout = 1u,   // an mbarrier wait exceeded its time limit
   kErrDrainTimeout = 2u,  // waiting for in-flight copies / MMAs at exit gave up
+  kErrBadLength = 4u,     // (debug builds) a sequence length outside [0, capacity]
+  kErrBadIndex = 8u,      // (debug builds) a selected index outside [0, L - recent), or unsorted
 };
 
-// Wall-clock limit for any single wait inside a kernel (nanoseconds).
-constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
+// Wall-clock limit for a wait on work in progress (nanoseconds): 2 s. A test build sets
+// MIMO_WAIT_LIMIT_NS to a few nanoseconds so that waits give up and the abort path runs.
+#ifndef MIMO_WAIT_LIMIT_NS
+#define MIMO_WAIT_LIMIT_NS 2000000000ull
+#endif
+constexpr unsigned long long kWaitLimitNs = MIMO_WAIT_LIMIT_NS;
+// Limit for the exit-path waits on copies and MMAs already in flight; always 2 s, so that a
+// CTA never leaves while an asynchronous copy may still write its shared memory.
+constexpr unsigned long long kDrainLimitNs = 2000000000ull;
 
 __device__ __forceinline__ unsigned long long globaltimer_ns() {
   unsigned long long t;
@@ -101,7 +110,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 __device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, unsigned* err) {
   const unsigned long long t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity)) {
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > kDrainLimitNs) {
       atomicOr(err, kErrDrainTimeout);
       return false;
     }

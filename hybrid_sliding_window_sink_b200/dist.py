@@ -35,6 +35,14 @@ def shard_range(n_units: int, rank: int, world: int) -> tuple[int, int]:
     return lo, lo + base + (1 if rank < extra else 0)
 
 
+def unit_shard(batch: int, n_kv_heads: int, rank: int, world: int) -> list[tuple[int, int]]:
+    """This rank's (sequence, KV head) units of a decode call: a contiguous block of the
+    flattened (b, g) order. Units share nothing, so a rank computes its block alone: the
+    query heads of KV head g, its cache rows and its outputs (the partition is exact)."""
+    lo, hi = shard_range(batch * n_kv_heads, rank, world)
+    return [divmod(u, n_kv_heads) for u in range(lo, hi)]
+
+
 def barrier():
     if dist.is_initialized():
         dist.barrier()

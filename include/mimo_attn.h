@@ -57,7 +57,7 @@ typedef enum mimo_status {
   MIMO_ERR_ALIGN = 4,       /* a data pointer is not 16-byte aligned */
   MIMO_ERR_WORKSPACE = 5,   /* workspace NULL or smaller than mimo_attn_workspace_size() */
   MIMO_ERR_CUDA = 6,        /* a CUDA call failed (no device, launch failure, ...) */
-  MIMO_ERR_DEVICE = 7       /* a kernel reported an internal timeout (see mimo_attn_last_device_error) */
+  MIMO_ERR_DEVICE = 7       /* a kernel set the device error word (see mimo_attn_device_status) */
 } mimo_status;
 
 /* Problem sizes. softmax_scale <= 0 selects 1/sqrt(head_dim_qk). */
@@ -346,9 +346,19 @@ mimo_status mimo_attn_check_indices(const mimo_shape* shape, const int* lengths,
                                     void* stream);
 
 /* Synchronises the current device, then returns and clears the device error word
- * that kernels set when a bounded wait gives up (0 = none). Host-blocking; for tests
- * and debugging. */
+ * (0 = none). Kernels OR bits into it instead of trapping: 1 = a wait on work in progress
+ * gave up (2 s; the kernel then left its loops, waited for its own copies and MMAs in flight,
+ * freed its tensor memory and returned without finishing its output), 2 = one of those
+ * exit-path waits gave up too, and in builds compiled with MIMO_DEBUG 4 = a sequence length
+ * outside [0, capacity] and 8 = a selected index outside [0, L - recent) or not increasing
+ * (both clamped, so no access leaves the caller's buffers). Host-blocking; for tests and
+ * debugging. Returns 0xFFFFFFFF if the device could not be synchronised. */
 unsigned int mimo_attn_last_device_error(void);
+
+/* mimo_attn_last_device_error as a status: MIMO_OK when the word was 0, MIMO_ERR_DEVICE
+ * when a kernel set it (the word is stored in *word when word is not NULL, then cleared),
+ * MIMO_ERR_CUDA when the device could not be synchronised. Host-blocking. */
+mimo_status mimo_attn_device_status(unsigned int* word);
 
 /* Static description of a status code. */
 const char* mimo_status_string(mimo_status status);
