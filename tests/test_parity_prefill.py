@@ -226,3 +226,26 @@ def test_full_size_sampled(cuda_device, case, nrand, heads):
     assert torch.isfinite(out).all() and torch.isfinite(lse).all()
     del inp, out, lse
     torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("B,n,hq,hkv,window,theta", [
+    (1, 700, 64, 8, 128, 1e4),     # SWA ring kernel: rotated K and V carried in f16
+    (1, 600, 64, 4, 0, 1e7),       # GA pair kernel: rotated K in f16
+    (1, 300, 16, 4, 64, 1e4),      # generic kernel
+])
+def test_large_magnitudes_inside_the_f16_range(cuda_device, B, n, hq, hkv, window, theta):
+    """K and V of magnitude in the thousands (Q scaled down so the logits keep their usual
+    size) pass through the kernels' f16 operands without clamping: the outputs, divided by
+    the V scale, and the lse match the oracle at the usual tolerances."""
+    inp = wl.prefill_inputs(B, n, hq, hkv, seed=77 + n)
+    q = (inp["q"].float() * 1e-3).to(torch.bfloat16)
+    k = (inp["k"].float() * 1e3).to(torch.bfloat16)
+    v = (inp["v"].float() * 2e3).to(torch.bfloat16)
+    assert float(k.float().abs().max()) > 3000 and float(v.float().abs().max()) > 6000
+    dev = cuda_device
+    out, lse = _lib.prefill(q.to(dev), k.to(dev), v.to(dev), inp["sink"].to(dev), window=window,
+                            rope_theta=theta, rot_dims=64)
+    torch.cuda.synchronize()
+    assert _lib.last_device_error() == 0
+    o_ref, l_ref = ref.prefill(wl.to_f64(q), wl.to_f64(k), wl.to_f64(v), wl.to_f64(inp["sink"]), window, theta, 64)
+    compare(wl.to_f64(out) / 2e3, o_ref / 2e3, wl.to_f64(lse), l_ref, f"large magnitudes W={window}")
