@@ -182,6 +182,25 @@ def timed_stream(fn, steps, warmup, stream):
         return timed(fn, steps, warmup, stream)
 
 
+def timed_graph(fn, steps, warmup, dev):
+    """Captures ``fn(stream)`` (launches on ``stream`` only) in a CUDA graph on a side stream and
+    times ``steps`` replays after ``warmup`` with CUDA events on that stream (``timed``). Short
+    kernels launched one by one from Python would otherwise be timed at the host's launch rate;
+    a serving loop replays its decode step as a graph, too."""
+    s = torch.cuda.Stream(device=dev)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(s):
+        fn(s)                        # outside capture first: library loaded, attributes set
+        s.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=s):
+            fn(s)
+    torch.cuda.synchronize()
+    ms = timed_stream(graph.replay, steps, warmup, s)
+    del graph
+    return ms
+
+
 def roofline_hbm(bytes_per_launch, ms_per_launch, peaks, tag, traffic=None):
     ach = bytes_per_launch / (ms_per_launch * 1e-3) / 1e9
     return {"bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -238,8 +257,8 @@ def bench_prefill(case, steps, warmup, peaks, tag, dev, stream, clocks=None):
 
 def bench_tiny_prefill(steps, peaks, tag, dev, stream):
     """Tiny SWA+sink prefill (n=1024, 8 Q / 1 KV, W=128): 5.9 MB of inputs and outputs, below
-    L2, so every launch is preceded by a 256 MB write that flushes L2 and is timed alone with
-    CUDA events on the launching stream."""
+    L2, so every launch follows a 256 MB write that flushes L2; the time is that of a CUDA
+    graph of (flush, prefill) minus that of a graph of the flush alone."""
     from hybrid_sliding_window_sink_b200 import _lib
     case = wl.TINY_SWA_PREFILL
     inp = wl.case_prefill_inputs(case, device=dev)
@@ -247,22 +266,15 @@ def bench_tiny_prefill(steps, peaks, tag, dev, stream):
     lse = torch.empty(case.batch, case.hq, case.seqlen, dtype=torch.float32, device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
-    def step():
+    def step(st):
         _lib.prefill(inp["q"], inp["k"], inp["v"], inp["sink"], window=case.window,
-                     rope_theta=case.theta, rot_dims=wl.ROT_DIMS, out=out, lse=lse, stream=stream)
+                     rope_theta=case.theta, rot_dims=wl.ROT_DIMS, out=out, lse=lse, stream=st)
 
-    for _ in range(3):
-        step()
-    torch.cuda.synchronize()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
-    with torch.cuda.stream(stream):
-        for e0, e1 in ev:
-            flush.fill_(1)
-            e0.record(stream)
-            step()
-            e1.record(stream)
-    torch.cuda.synchronize()
-    ms = statistics.median(e0.elapsed_time(e1) for e0, e1 in ev)
+    # graph(flush, prefill) minus graph(flush): the kernel's time after an L2 flush, without the
+    # host's launch latency
+    ms_both = timed_graph(lambda st: (flush.fill_(1), step(st)), steps, 3, dev) / steps
+    ms_flush = timed_graph(lambda st: flush.fill_(1), steps, 3, dev) / steps
+    ms = ms_both - ms_flush
     flops, bytes_ = prefill_work(case)
     del inp, out, lse, flush
     return {"ms": round(ms, 5), "tflops": round(flops / (ms * 1e-3) / 1e12, 2),
@@ -377,16 +389,12 @@ def bench_decode_step(steps, warmup, peaks, tag, dev, stream, batch_range=None):
                               kind=_lib.MIMO_CACHE_LINEAR, capacity=cg.capacity)
     ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
 
-    def run_layer(lay):
+    def run_layer(lay, st):
         kind, q, kc, vc, sink, out, lse = lay
         _lib.decode(q, kc, vc, Ld, sink, kind="ring" if kind == 1 else "linear",
-                    out=out, lse=lse, workspace=ws, stream=stream)
+                    out=out, lse=lse, workspace=ws, stream=st)
 
-    def step():
-        for lay in layers:
-            run_layer(lay)
-
-    ms = timed(step, steps, warmup, stream)
+    ms = timed_graph(lambda st: [run_layer(l, st) for l in layers], steps, warmup, dev)
     Ls = L.tolist()
     b_swa = decode_layer_bytes(Ls, cs.hq, cs.hkv, "ring", cs.capacity)
     b_ga = decode_layer_bytes(Ls, cg.hq, cg.hkv, "linear", cg.capacity)
@@ -394,12 +402,12 @@ def bench_decode_step(steps, warmup, peaks, tag, dev, stream, batch_range=None):
     # per-kind kernel time: time GA layers and SWA layers separately
     ga_layers = [l for l in layers if l[0] == 0]
     swa_layers = [l for l in layers if l[0] == 1]
-    ms_ga = timed(lambda: [run_layer(l) for l in ga_layers], steps, 1, stream) / (steps * 9)
-    ms_swa = timed(lambda: [run_layer(l) for l in swa_layers], steps, 1, stream) / (steps * 39)
+    ms_ga = timed_graph(lambda st: [run_layer(l, st) for l in ga_layers], steps, 1, dev) / (steps * 9)
+    ms_swa = timed_graph(lambda st: [run_layer(l, st) for l in swa_layers], steps, 1, dev) / (steps * 39)
     res = {
         "value": round(total / (ms / steps * 1e-3) / 1e9, 1), "unit": "GB/s",
         "ms_per_step": round(ms / steps, 4), "bytes_per_step": total,
-        "launches_per_step": 39 + 9 * 2,
+        "launches_per_step": 39 + 9 * 2, "graph": True,
         "ga_layer": roofline_hbm(b_ga, ms_ga, peaks, tag,
                                  traffic_for("decode_split_linear", int(sum(Ls)) * cg.hkv)),
         "swa_layer": roofline_hbm(b_swa, ms_swa, peaks, tag),
@@ -456,20 +464,20 @@ def bench_mtp_step(steps, warmup, peaks, tag, dev, stream, q_len=4):
                                                             cg.capacity, q_len, 0))
     ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
 
-    def run_layer(lay):
+    def run_layer(lay, st):
         kind, q, kc, vc, sink, out, lse = lay
         _lib.decode_mq(q, kc, vc, Ld, sink, kind="ring" if kind == 1 else "linear",
-                       window=wl.SWA_WINDOW, out=out, lse=lse, workspace=ws, stream=stream)
+                       window=wl.SWA_WINDOW, out=out, lse=lse, workspace=ws, stream=st)
 
-    ms = timed(lambda: [run_layer(l) for l in layers], steps, warmup, stream)
+    ms = timed_graph(lambda st: [run_layer(l, st) for l in layers], steps, warmup, dev)
     Ls = L.tolist()
     b_swa = mtp_layer_bytes(Ls, cs.hq, cs.hkv, "ring", cap_ring, q_len)
     b_ga = mtp_layer_bytes(Ls, cg.hq, cg.hkv, "linear", cg.capacity, q_len)
     total = 39 * b_swa + 9 * b_ga
     ga_layers = [l for l in layers if l[0] == 0]
     swa_layers = [l for l in layers if l[0] == 1]
-    ms_ga = timed(lambda: [run_layer(l) for l in ga_layers], steps, 1, stream) / (steps * 9)
-    ms_swa = timed(lambda: [run_layer(l) for l in swa_layers], steps, 1, stream) / (steps * 39)
+    ms_ga = timed_graph(lambda st: [run_layer(l, st) for l in ga_layers], steps, 1, dev) / (steps * 9)
+    ms_swa = timed_graph(lambda st: [run_layer(l, st) for l in swa_layers], steps, 1, dev) / (steps * 39)
     flops_ga = 2.0 * (wl.DQK + wl.DV) * q_len * cg.hq * float(np.sum(Ls))   # upper bound: all keys
     res = {
         "value": round(total / (ms / steps * 1e-3) / 1e9, 1), "unit": "GB/s",
@@ -528,18 +536,18 @@ def bench_fp8_decode_step(steps, warmup, peaks, tag, dev, stream):
                               kind=_lib.MIMO_CACHE_LINEAR, capacity=cg.capacity)
     ws = torch.empty(max(nws, 16), dtype=torch.uint8, device=dev)
 
-    def run_layer(lay):
+    def run_layer(lay, st):
         kind, q, (k8, v8, ks, vs), sink, out, lse = lay
         _lib.decode_fp8(q, k8, v8, ks, vs, Ld, sink, kind="ring" if kind == 1 else "linear",
-                        out=out, lse=lse, workspace=ws, stream=stream)
+                        out=out, lse=lse, workspace=ws, stream=st)
 
-    ms = timed(lambda: [run_layer(l) for l in layers], steps, warmup, stream)
+    ms = timed_graph(lambda st: [run_layer(l, st) for l in layers], steps, warmup, dev)
     Ls = L.tolist()
     b_swa = fp8_decode_layer_bytes(Ls, cs.hq, cs.hkv, "ring", cs.capacity)
     b_ga = fp8_decode_layer_bytes(Ls, cg.hq, cg.hkv, "linear", cg.capacity)
     total = 39 * b_swa + 9 * b_ga
-    ms_ga = timed(lambda: [run_layer(l) for l in layers if l[0] == 0], steps, 1, stream) / (steps * 9)
-    ms_swa = timed(lambda: [run_layer(l) for l in layers if l[0] == 1], steps, 1, stream) / (steps * 39)
+    ms_ga = timed_graph(lambda st: [run_layer(l, st) for l in layers if l[0] == 0], steps, 1, dev) / (steps * 9)
+    ms_swa = timed_graph(lambda st: [run_layer(l, st) for l in layers if l[0] == 1], steps, 1, dev) / (steps * 39)
     res = {
         "value": round(total / (ms / steps * 1e-3) / 1e9, 1), "unit": "GB/s",
         "ms_per_step": round(ms / steps, 4), "bytes_per_step": total,

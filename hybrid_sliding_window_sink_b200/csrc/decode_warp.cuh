@@ -31,101 +31,55 @@ constexpr int kDwMaxStages = 3;
 
 __host__ __device__ constexpr int dw_smem_bytes(int stages) { return stages * (kDwStageBytes + kDwKeys * 4); }
 
-template <int G, int NS>
-__global__ void __launch_bounds__(32) decode_warp_kernel(const DecodeParams p) {
-  static_assert(G >= 1 && G <= 16, "group size");
-  static_assert(NS >= 1 && NS <= kDwMaxStages, "stages in flight");
-  extern __shared__ __align__(1024) uint8_t smem[];
-  const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-  const int lane = threadIdx.x, gq = lane >> 2, tq = lane & 3;
-
-  int nw, L;
-  const int nkeys = dec_unit_keys(p, b, nw, L);
-  const int k_begin = c * p.chunk;
-  int n_here = nkeys - k_begin;
-  n_here = n_here < 0 ? 0 : (n_here < p.chunk ? n_here : p.chunk);
-  if (n_here == 0 && !p.direct) return;          // empty chunk: the combine skips it
-
-  const uint32_t s_base = smem_u32(smem);
-  int* s_tok = reinterpret_cast<int*>(smem + NS * kDwStageBytes);   // [NS][32]
-  const int nst = (n_here + kDwKeys - 1) / kDwKeys;
-  const long long seq0 = static_cast<long long>(b) * p.seq_stride;
-  const __nv_bfloat16* kbase = p.k + g * kDQK;
-  const __nv_bfloat16* vbase = p.v + g * kDV;
-  const long long krow_stride = static_cast<long long>(p.Hkv) * kDQK;
-  const long long vrow_stride = static_cast<long long>(p.Hkv) * kDV;
-
-  // Gathers stage st (keys 32 st .. 32 st + 31 of the chunk) into buffer st % NS: each lane
-  // resolves the token of its own key (-1 when masked), then the warp copies the 32 rows
-  // 16 bytes per lane and instruction.
-  auto issue = [&](int st, int tok) {
-    const int buf = st % NS;
-    int* tk = s_tok + buf * kDwKeys;
-    tk[lane] = tok;
-    __syncwarp();
-    const uint32_t sK = s_base + buf * kDwStageBytes;
-    const uint32_t sV = sK + kDwKeys * kKRow;
+// The warp copies 32 K and V rows (tokens tk[0..31] of one sequence and KV head; a negative
+// token is zero-filled) into a stage by 16-byte cp.async: 24 + 16 chunks per lane, K rows
+// XOR-swizzled for ldmatrix. The caller commits the group.
+__device__ __forceinline__ void dw_gather(uint32_t sK, uint32_t sV, const int* tk, const __nv_bfloat16* kbase,
+                                          const __nv_bfloat16* vbase, long long seq0, long long krow_stride,
+                                          long long vrow_stride) {
+  const int lane = threadIdx.x & 31;
 #pragma unroll 8
-    for (int i = 0; i < 24; ++i) {                 // 32 rows x 24 chunks of K
-      const int idx = lane + 32 * i;
-      const int row = idx / 24, u = idx - row * 24;
-      const int t = tk[row];
-      cp_async16(sK + row * kKRow + ((u ^ (row & 7)) << 4),
-                 kbase + (seq0 + (t < 0 ? 0 : t)) * krow_stride + u * 8, t < 0 ? 0u : 16u);
-    }
+  for (int i = 0; i < 24; ++i) {                   // 32 rows x 24 chunks of K
+    const int idx = lane + 32 * i;
+    const int row = idx / 24, u = idx - row * 24;
+    const int t = tk[row];
+    cp_async16(sK + row * kKRow + ((u ^ (row & 7)) << 4),
+               kbase + (seq0 + (t < 0 ? 0 : t)) * krow_stride + u * 8, t < 0 ? 0u : 16u);
+  }
 #pragma unroll 8
-    for (int i = 0; i < 16; ++i) {                 // 32 rows x 16 chunks of V
-      const int idx = lane + 32 * i;
-      const int row = idx >> 4, u = idx & 15;
-      const int t = tk[row];
-      cp_async16(sV + row * kVRow + ((u ^ (row & 7)) << 4),
-                 vbase + (seq0 + (t < 0 ? 0 : t)) * vrow_stride + u * 8, t < 0 ? 0u : 16u);
-    }
-  };
-  auto token = [&](int st) -> int {
-    const int key = st * kDwKeys + lane;
-    return key < n_here ? dec_token(p, b, g, k_begin + key, nw, L) : -1;
-  };
-  {
-    int tok[NS];
-#pragma unroll
-    for (int s = 0; s < NS; ++s) tok[s] = s < nst ? token(s) : -1;   // index loads all in flight
-#pragma unroll
-    for (int s = 0; s < NS; ++s) {
-      if (s < nst) issue(s, tok[s]);
-      cp_async_commit();
-    }
+  for (int i = 0; i < 16; ++i) {                   // 32 rows x 16 chunks of V
+    const int idx = lane + 32 * i;
+    const int row = idx >> 4, u = idx & 15;
+    const int t = tk[row];
+    cp_async16(sV + row * kVRow + ((u ^ (row & 7)) << 4),
+               vbase + (seq0 + (t < 0 ? 0 : t)) * vrow_stride + u * 8, t < 0 ? 0u : 16u);
   }
+}
 
-  // Query fragments (A operand, rows = the group's heads, zero-padded to 16).
-  uint32_t qa[12][4];
-  {
-    const __nv_bfloat16* qg = p.q + (static_cast<long long>(b) * p.Hq + g * G) * kDQK;
-    const bool r0ok = gq < G, r1ok = gq + 8 < G;
+// Query fragments of the group's G heads (rows gq, gq + 8 of the m16 A operand; padding
+// rows are zero), read once per warp from q [G, 192].
+template <int G>
+__device__ __forceinline__ void dw_load_q(uint32_t (&qa)[12][4], const __nv_bfloat16* qg) {
+  const int lane = threadIdx.x & 31, gq = lane >> 2, tq = lane & 3;
+  const bool r0ok = gq < G, r1ok = gq + 8 < G;
 #pragma unroll
-    for (int kk = 0; kk < 12; ++kk) {
-      const int d0 = kk * 16 + tq * 2;
-      qa[kk][0] = r0ok ? __ldg(reinterpret_cast<const unsigned*>(qg + gq * kDQK + d0)) : 0u;
-      qa[kk][1] = r1ok ? __ldg(reinterpret_cast<const unsigned*>(qg + (gq + 8) * kDQK + d0)) : 0u;
-      qa[kk][2] = r0ok ? __ldg(reinterpret_cast<const unsigned*>(qg + gq * kDQK + d0 + 8)) : 0u;
-      qa[kk][3] = r1ok ? __ldg(reinterpret_cast<const unsigned*>(qg + (gq + 8) * kDQK + d0 + 8)) : 0u;
-    }
+  for (int kk = 0; kk < 12; ++kk) {
+    const int d0 = kk * 16 + tq * 2;
+    qa[kk][0] = r0ok ? __ldg(reinterpret_cast<const unsigned*>(qg + gq * kDQK + d0)) : 0u;
+    qa[kk][1] = r1ok ? __ldg(reinterpret_cast<const unsigned*>(qg + (gq + 8) * kDQK + d0)) : 0u;
+    qa[kk][2] = r0ok ? __ldg(reinterpret_cast<const unsigned*>(qg + gq * kDQK + d0 + 8)) : 0u;
+    qa[kk][3] = r1ok ? __ldg(reinterpret_cast<const unsigned*>(qg + (gq + 8) * kDQK + d0 + 8)) : 0u;
   }
+}
 
-  float o[16][4];
-#pragma unroll
-  for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+// One stage of 32 keys for one warp: S = Q K^T (K rows XOR-swizzled at sK), the online
+// softmax in the log2 domain (a key whose token tk[key] < 0 is masked), and O += P V (V rows at
+// sV). m0 / m1 and l0 / l1 are this thread's running max and (partial) sum of rows gq, gq + 8.
+__device__ __forceinline__ void dw_stage(uint32_t sK, uint32_t sV, const int* tk, const uint32_t (&qa)[12][4],
+                                         float scale_log2, float (&o)[16][4], float& m0, float& m1,
+                                         float& l0, float& l1) {
+  const int lane = threadIdx.x & 31, tq = lane & 3;
   const int mi = lane >> 3, r8 = lane & 7;
-
-  for (int st = 0; st < nst; ++st) {
-    const int buf = st % NS;
-    cp_async_wait<NS - 1>();                       // this lane's copies of stage st have landed
-    __syncwarp();                                  // ... and every other lane's
-    const int* tk = s_tok + buf * kDwKeys;
-    const uint32_t sK = s_base + buf * kDwStageBytes;
-    const uint32_t sV = sK + kDwKeys * kKRow;
-
     // S = Q K^T for the stage's 32 keys: four n-tiles of 8 keys.
     float sacc[4][4];
 #pragma unroll
@@ -149,7 +103,7 @@ __global__ void __launch_bounds__(32) decode_warp_kernel(const DecodeParams p) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int key = nt * 8 + tq * 2 + (e & 1);
-        s[nt][e] = tk[key] >= 0 ? sacc[nt][e] * p.scale_log2 : -INFINITY;
+        s[nt][e] = tk[key] >= 0 ? sacc[nt][e] * scale_log2 : -INFINITY;
       }
     float mx0 = fmaxf(fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1])),
                       fmaxf(fmaxf(s[2][0], s[2][1]), fmaxf(s[3][0], s[3][1])));
@@ -201,6 +155,75 @@ __global__ void __launch_bounds__(32) decode_warp_kernel(const DecodeParams p) {
         mma_16816(o[2 * jp + 1], pa, v2, v3);
       }
     }
+}
+
+template <int G, int NS>
+__global__ void __launch_bounds__(32) decode_warp_kernel(const DecodeParams p) {
+  static_assert(G >= 1 && G <= 16, "group size");
+  static_assert(NS >= 1 && NS <= kDwMaxStages, "stages in flight");
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int lane = threadIdx.x, gq = lane >> 2, tq = lane & 3;
+
+  int nw, L;
+  const int nkeys = dec_unit_keys(p, b, nw, L);
+  const int k_begin = c * p.chunk;
+  int n_here = nkeys - k_begin;
+  n_here = n_here < 0 ? 0 : (n_here < p.chunk ? n_here : p.chunk);
+  if (n_here == 0 && !p.direct) return;          // empty chunk: the combine skips it
+
+  const uint32_t s_base = smem_u32(smem);
+  int* s_tok = reinterpret_cast<int*>(smem + NS * kDwStageBytes);   // [NS][32]
+  const int nst = (n_here + kDwKeys - 1) / kDwKeys;
+  const long long seq0 = static_cast<long long>(b) * p.seq_stride;
+  const __nv_bfloat16* kbase = p.k + g * kDQK;
+  const __nv_bfloat16* vbase = p.v + g * kDV;
+  const long long krow_stride = static_cast<long long>(p.Hkv) * kDQK;
+  const long long vrow_stride = static_cast<long long>(p.Hkv) * kDV;
+
+  // Gathers stage st (keys 32 st .. 32 st + 31 of the chunk) into buffer st % NS: each lane
+  // resolves the token of its own key (-1 when masked), then the warp copies the 32 rows.
+  auto issue = [&](int st, int tok) {
+    const int buf = st % NS;
+    int* tk = s_tok + buf * kDwKeys;
+    tk[lane] = tok;
+    __syncwarp();
+    const uint32_t sK = s_base + buf * kDwStageBytes;
+    dw_gather(sK, sK + kDwKeys * kKRow, tk, kbase, vbase, seq0, krow_stride, vrow_stride);
+  };
+  auto token = [&](int st) -> int {
+    const int key = st * kDwKeys + lane;
+    return key < n_here ? dec_token(p, b, g, k_begin + key, nw, L) : -1;
+  };
+  {
+    int tok[NS];
+#pragma unroll
+    for (int s = 0; s < NS; ++s) tok[s] = s < nst ? token(s) : -1;   // index loads all in flight
+#pragma unroll
+    for (int s = 0; s < NS; ++s) {
+      if (s < nst) issue(s, tok[s]);
+      cp_async_commit();
+    }
+  }
+
+  // Query fragments (A operand, rows = the group's heads, zero-padded to 16).
+  uint32_t qa[12][4];
+  dw_load_q<G>(qa, p.q + (static_cast<long long>(b) * p.Hq + g * G) * kDQK);
+
+  float o[16][4];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+
+  for (int st = 0; st < nst; ++st) {
+    const int buf = st % NS;
+    cp_async_wait<NS - 1>();                       // this lane's copies of stage st have landed
+    __syncwarp();                                  // ... and every other lane's
+    const int* tk = s_tok + buf * kDwKeys;
+    const uint32_t sK = s_base + buf * kDwStageBytes;
+    const uint32_t sV = sK + kDwKeys * kKRow;
+
+    dw_stage(sK, sV, tk, qa, p.scale_log2, o, m0, m1, l0, l1);
     __syncwarp();                                  // every lane is done reading the buffer
     if (st + NS < nst) issue(st + NS, token(st + NS));
     cp_async_commit();
