@@ -31,55 +31,6 @@
 
 namespace mimo {
 
-// max of three floats in one instruction (sm_100 three-input max).
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-  float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
-
-// Two floats -> packed f16x2, round to nearest even, saturating to the finite f16 range.
-__device__ __forceinline__ uint32_t pack_f16_satfinite(float lo, float hi) {
-  uint32_t r;
-  asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-
-// Packed f32x2 arithmetic (two fp32 lanes per 64-bit register pair, rounded per lane).
-// Volatile: its inputs come from tcgen05.ld, so it stays after the wait::ld that follows the
-// load (volatile asm statements keep their order).
-__device__ __forceinline__ unsigned long long ga_f2_bits(uint32_t lo, uint32_t hi) {
-  unsigned long long r;
-  asm volatile("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
-  return r;
-}
-__device__ __forceinline__ unsigned long long ga_f2_pack(float lo, float hi) {
-  unsigned long long r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ float2 ga_f2_unpack(unsigned long long x) {
-  float2 r;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(x));
-  return r;
-}
-__device__ __forceinline__ unsigned long long ga_f2_fma(unsigned long long a, unsigned long long b,
-                                                        unsigned long long c) {
-  unsigned long long r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-  return r;
-}
-__device__ __forceinline__ unsigned long long ga_f2_add(unsigned long long a, unsigned long long b) {
-  unsigned long long r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-__device__ __forceinline__ unsigned long long ga_f2_mul(unsigned long long a, unsigned long long b) {
-  unsigned long long r;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-
 // 32 consecutive TMEM columns of this warp's 32 lanes.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   tmem_ld16(taddr, *reinterpret_cast<uint32_t(*)[16]>(r));
@@ -436,8 +387,8 @@ __global__ void __launch_bounds__(kGaThreads, 1)
                     r1[h] = x1 * c - x2 * sn;
                     r2[h] = x2 * c + x1 * sn;
                   }
-                  xs[e2] = pack_f16_satfinite(r1[0], r1[1]);
-                  ys[e2] = pack_f16_satfinite(r2[0], r2[1]);
+                  xs[e2] = pack_f16_sat(r1[0], r1[1]);
+                  ys[e2] = pack_f16_sat(r2[0], r2[1]);
                 }
                 *px = make_uint4(xs[0], xs[1], xs[2], xs[3]);
                 *py = make_uint4(ys[0], ys[1], ys[2], ys[3]);
@@ -530,9 +481,9 @@ __global__ void __launch_bounds__(kGaThreads, 1)
         }
         const float ref = m == -INFINITY ? 0.f : m;
         // pass 2: P = 2^(a - ref) (0 above the diagonal), bf16 into S columns [0, 64)
-        const unsigned long long sc2 = ga_f2_pack(p.scale_log2, p.scale_log2);
-        const unsigned long long nref2 = ga_f2_pack(-ref, -ref);
-        unsigned long long sab = ga_f2_pack(0.f, 0.f);   // row sums of even and odd columns
+        const unsigned long long sc2 = f2_pack(p.scale_log2, p.scale_log2);
+        const unsigned long long nref2 = f2_pack(-ref, -ref);
+        unsigned long long sab = f2_pack(0.f, 0.f);   // row sums of even and odd columns
         auto pass2 = [&](auto masked) {
 #pragma unroll 1
           for (int c = 0; c < kGaBN; c += 64) {
@@ -549,14 +500,14 @@ __global__ void __launch_bounds__(kGaThreads, 1)
 #pragma unroll
               for (int e = 0; e < 8; ++e) {
                 const int col = 16 * q + 2 * e;
-                const float2 y = ga_f2_unpack(ga_f2_fma(ga_f2_bits(v[col], v[col + 1]), sc2, nref2));
+                const float2 y = f2_unpack(f2_fma(f2_bits(v[col], v[col + 1]), sc2, nref2));
                 float a0 = ex2(y.x);
                 float a1 = ex2(y.y);
                 if (decltype(masked)::value) {
                   a0 = col <= lim ? a0 : 0.f;
                   a1 = col + 1 <= lim ? a1 : 0.f;
                 }
-                sab = ga_f2_add(sab, ga_f2_pack(a0, a1));
+                sab = f2_add(sab, f2_pack(a0, a1));
                 pk[e] = pack_bf16(a0, a1);
               }
               tmem_st8(trow + (c >> 1) + 8 * q, pk);
@@ -570,7 +521,7 @@ __global__ void __launch_bounds__(kGaThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(kGaPReady + grp));
-        const float2 s2 = ga_f2_unpack(sab);
+        const float2 s2 = f2_unpack(sab);
         l += s2.x + s2.y;
       }
       if (!ok) break;
@@ -587,11 +538,11 @@ __global__ void __launch_bounds__(kGaThreads, 1)
         tmem_wait_ld();
         if (row_ok) {
           uint32_t pk[16];
-          const unsigned long long il2 = ga_f2_pack(inv_l, inv_l);
+          const unsigned long long il2 = f2_pack(inv_l, inv_l);
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const float2 o0 = ga_f2_unpack(ga_f2_mul(ga_f2_bits(v0[2 * e], v0[2 * e + 1]), il2));
-            const float2 o1 = ga_f2_unpack(ga_f2_mul(ga_f2_bits(v1[2 * e], v1[2 * e + 1]), il2));
+            const float2 o0 = f2_unpack(f2_mul(f2_bits(v0[2 * e], v0[2 * e + 1]), il2));
+            const float2 o1 = f2_unpack(f2_mul(f2_bits(v1[2 * e], v1[2 * e + 1]), il2));
             pk[e] = pack_bf16(o0.x, o0.y);
             pk[8 + e] = pack_bf16(o1.x, o1.y);
           }

@@ -103,46 +103,6 @@ enum : int {
   kSwNumBars = 50
 };
 
-// Packed f32x2 helpers (two fp32 lanes in one 64-bit register pair, rounded per lane).
-// Volatile: its inputs come from tcgen05.ld, so it must stay after the wait::ld that follows
-// the load (volatile asm statements keep their order).
-__device__ __forceinline__ unsigned long long f2_bits(uint32_t lo, uint32_t hi) {
-  unsigned long long r;
-  asm volatile("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
-  return r;
-}
-__device__ __forceinline__ unsigned long long f2_pack(float lo, float hi) {
-  unsigned long long r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ float2 f2_unpack(unsigned long long x) {
-  float2 r;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(x));
-  return r;
-}
-__device__ __forceinline__ unsigned long long f2_fma(unsigned long long a, unsigned long long b,
-                                                     unsigned long long c) {
-  unsigned long long r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-  return r;
-}
-__device__ __forceinline__ unsigned long long f2_add(unsigned long long a, unsigned long long b) {
-  unsigned long long r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-__device__ __forceinline__ unsigned long long f2_mul(unsigned long long a, unsigned long long b) {
-  unsigned long long r;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-__device__ __forceinline__ float swa_max3(float a, float b, float c) {   // volatile: see f2_bits
-  float r;
-  asm volatile("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
-
 // (x, y) <- (x cos - y sin, y cos + x sin) for two rotation pairs: xw and yw each hold two
 // bf16 (dims k, k+1 of the first and of the second half), cs = (cos k, cos k+1, sin k,
 // sin k+1). Packed f32x2 arithmetic, results rounded to f16 with clamping.
@@ -546,8 +506,8 @@ __global__ void __launch_bounds__(kSwaThreads, 1)
             float mb = -INFINITY;
 #pragma unroll
             for (int e = 0; e < 16; e += 4) {
-              mq = swa_max3(mq, __uint_as_float(v[q][e]), __uint_as_float(v[q][e + 1]));
-              mb = swa_max3(mb, __uint_as_float(v[q][e + 2]), __uint_as_float(v[q][e + 3]));
+              mq = fmax3_v(mq, __uint_as_float(v[q][e]), __uint_as_float(v[q][e + 1]));
+              mb = fmax3_v(mb, __uint_as_float(v[q][e + 2]), __uint_as_float(v[q][e + 3]));
             }
             mq = fmaxf(mq, mb);
           } else if (k[q] == 1) {

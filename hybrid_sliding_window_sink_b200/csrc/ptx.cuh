@@ -269,7 +269,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
-// Two floats -> packed f16x2 (round to nearest even), clamped to the finite f16 range.
 // Round to f16 with values beyond the f16 range clamped to +-65504 (one cvt with satfinite).
 __device__ __forceinline__ uint32_t pack_f16_sat(float lo, float hi) {
   uint32_t r;
@@ -280,6 +279,54 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
   __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
+// Packed f32x2 arithmetic: two fp32 lanes in one 64-bit register pair, each lane rounded on
+// its own. f2_bits is volatile: its inputs come from tcgen05.ld, so it has to stay after the
+// tcgen05.wait::ld that follows the load (volatile asm statements keep their order).
+__device__ __forceinline__ unsigned long long f2_bits(uint32_t lo, uint32_t hi) {
+  unsigned long long r;
+  asm volatile("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+  return r;
+}
+__device__ __forceinline__ unsigned long long f2_pack(float lo, float hi) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 f2_unpack(unsigned long long x) {
+  float2 r;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(x));
+  return r;
+}
+__device__ __forceinline__ unsigned long long f2_fma(unsigned long long a, unsigned long long b,
+                                                     unsigned long long c) {
+  unsigned long long r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ unsigned long long f2_add(unsigned long long a, unsigned long long b) {
+  unsigned long long r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ unsigned long long f2_mul(unsigned long long a, unsigned long long b) {
+  unsigned long long r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// Max of three floats in one instruction (sm_100 three-input max). fmax3_v is the volatile
+// form for operands that come straight from tcgen05.ld (see f2_bits).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ float fmax3_v(float a, float b, float c) {
+  float r;
+  asm volatile("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // Packed bf16 pair -> packed f16 pair (exact inside the f16 range, clamped outside it).
 __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t v) {
   return pack_f16_sat(__uint_as_float(v << 16), __uint_as_float(v & 0xFFFF0000u));
