@@ -410,7 +410,8 @@ def bench_decode_step(steps, warmup, peaks, tag, dev, stream, batch_range=None):
         "launches_per_step": 39 + 9 * 2, "graph": True,
         "ga_layer": roofline_hbm(b_ga, ms_ga, peaks, tag,
                                  traffic_for("decode_split_linear", int(sum(Ls)) * cg.hkv)),
-        "swa_layer": roofline_hbm(b_swa, ms_swa, peaks, tag),
+        "swa_layer": roofline_hbm(b_swa, ms_swa, peaks, tag,      # every ring is full (L >= 4096)
+                                  traffic_for("decode_warp_ring", len(Ls) * cs.hkv)),
         "roofline": roofline_hbm(total, ms / steps, peaks, tag),
         "ms_ga_layer": round(ms_ga, 4), "ms_swa_layer": round(ms_swa, 5),
         "cache": "39 distinct SWA ring caches; one padded GA cache [64,131072,4,*] read by all 9 GA layers",
@@ -553,7 +554,7 @@ def bench_fp8_decode_step(steps, warmup, peaks, tag, dev, stream):
         "ms_per_step": round(ms / steps, 4), "bytes_per_step": total,
         "launches_per_step": 39 + 9 * 2,
         "ga_layer": roofline_hbm(b_ga, ms_ga, peaks, tag,
-                                 traffic_for("decode_split_fp8_linear", int(sum(Ls)) * cg.hkv)),
+                                 traffic_for("decode_fp8_linear", int(sum(Ls)) * cg.hkv)),
         "swa_layer": roofline_hbm(b_swa, ms_swa, peaks, tag),
         "roofline": roofline_hbm(total, ms / steps, peaks, tag),
         "ms_ga_layer": round(ms_ga, 4), "ms_swa_layer": round(ms_swa, 5),
@@ -645,7 +646,7 @@ def bench_sparse(steps, warmup, peaks, tag, dev, stream, calls=16):
            "ms_per_call": round(ms_call, 5), "bytes_per_call": per_call_bytes, "calls_per_step": calls,
            "launches_per_call": 2,
            "roofline": roofline_hbm(per_call_bytes, ms_call, peaks, tag,
-                                    traffic_for("decode_split_sparse", c.batch * c.hkv)),
+                                    traffic_for("decode_warp_sparse", c.batch * c.hkv)),
            "graph": True}
     del graph, sets, base
     return res

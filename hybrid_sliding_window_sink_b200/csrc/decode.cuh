@@ -23,12 +23,7 @@
 // group's (up to 16) query heads as the M dimension; online softmax per warp; the
 // four warp states are merged at the end.
 //
-// FP8 caches (FP8 = true): K and V rows are OCP E4M3 bytes with one fp32 scale per (token,
-// KV head) row for each tensor. Each subtile's bytes and scales are gathered by cp.async
-// into a raw stage, then converted exactly into the MMA layout: K to f16 (E4M3 -> f16 is
-// exact) for an f16 S = Q K^T with Q converted to f16 once, V to bf16 (exact). The K scale
-// multiplies the fp32 score; the V scale multiplies P before it is rounded to bf16 for the
-// PV MMA, while the denominator sums the unscaled P. Q must lie inside the f16 range.
+// FP8 caches have kernels of their own (decode_fp8.cuh).
 #pragma once
 
 #include "ptx.cuh"
@@ -45,10 +40,7 @@ constexpr int kVRow = kDV * 2;                     // 256 bytes
 constexpr int kDecStageBytes = kDecSub * (kKRow + kVRow);   // 40960
 constexpr int kDecMaxTokList = 512;                // sparse chunk limit (tokens staged in smem)
 constexpr int kDecSmemBytes = kDecStages * kDecStageBytes + kDecMaxTokList * 4;
-// FP8: one converted stage, two raw stages (bytes + scales), per-subtile scales, token list
-constexpr int kKRow8 = kDQK, kVRow8 = kDV;                    // bytes per cached row
-constexpr int kDecRawBytes = kDecSub * (kKRow8 + kVRow8) + 2 * kDecSub * 4;   // 20992
-constexpr int kDecSmemBytesFp8 = kDecStageBytes + 2 * kDecRawBytes + 2 * kDecSub * 4 + kDecMaxTokList * 4;
+constexpr int kKRow8 = kDQK, kVRow8 = kDV;                    // FP8 bytes per cached row
 
 enum : int { kModeRing = 0, kModeLinear = 1, kModeSparse = 2 };
 
@@ -131,16 +123,12 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
   asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
   return r;
 }
-// Packed f16x2 holding E4M3 values (at most 4 significant bits) -> packed bf16x2, exactly.
-__device__ __forceinline__ uint32_t f16x2_to_bf16x2(uint32_t v) {
-  const __half2 h = *reinterpret_cast<const __half2*>(&v);
-  const float2 f = __half22float2(h);
-  return pack_bf16(f.x, f.y);
-}
 
-template <int G, bool FP8 = false>
+template <int G>
 __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const DecodeParams p) {
   static_assert(G >= 1 && G <= 16, "group size");
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(1024) uint8_t smem[];
   const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -153,8 +141,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
   int n_here = nkeys - k_begin;
   n_here = n_here < 0 ? 0 : (n_here < p.chunk ? n_here : p.chunk);
 
-  int* s_tok = reinterpret_cast<int*>(smem + (FP8 ? kDecSmemBytesFp8 - kDecMaxTokList * 4
-                                                    : kDecStages * kDecStageBytes));
+  int* s_tok = reinterpret_cast<int*>(smem + kDecStages * kDecStageBytes);
   if (p.mode == kModeSparse) {
     for (int i = tid; i < n_here; i += kDecThreads) s_tok[i] = dec_token(p, b, g, k_begin + i, nw, L);
     __syncthreads();
@@ -170,49 +157,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
     return p.mode == kModeSparse ? s_tok[key] : k_begin + key;
   };
 
-  const uint8_t* kbase8 = p.k8 + g * kKRow8;
-  const uint8_t* vbase8 = p.v8 + g * kVRow8;
-  // FP8: bytes and scales of subtile st into raw stage `stage` (unswizzled rows)
-  auto load_raw = [&](int st, int stage) {
-    const uint32_t r0 = s_base + kDecStageBytes + stage * kDecRawBytes;
-    const uint32_t rK = r0, rV = r0 + kDecSub * kKRow8, rS = rV + kDecSub * kVRow8;
-    const int base = st * kDecSub;
-#pragma unroll
-    for (int i = 0; i < (kDecSub * 12) / kDecThreads; ++i) {      // 6 x 16 B of K per thread
-      const int idx = tid + i * kDecThreads;
-      const int row = idx / 12, u = idx - row * 12;
-      const int key = base + row;
-      int tok = key < n_here ? token_of(key) : -1;
-      const bool ok = tok >= 0;
-      tok = ok ? tok : 0;
-      cp_async16(rK + row * kKRow8 + u * 16, kbase8 + (seq0 + tok) * (krow_stride) + u * 16, ok ? 16u : 0u);
-    }
-#pragma unroll
-    for (int i = 0; i < (kDecSub * 8) / kDecThreads; ++i) {       // 4 x 16 B of V per thread
-      const int idx = tid + i * kDecThreads;
-      const int row = idx >> 3, u = idx & 7;
-      const int key = base + row;
-      int tok = key < n_here ? token_of(key) : -1;
-      const bool ok = tok >= 0;
-      tok = ok ? tok : 0;
-      cp_async16(rV + row * kVRow8 + u * 16, vbase8 + (seq0 + tok) * (vrow_stride) + u * 16, ok ? 16u : 0u);
-    }
-    {                                                             // one scale per thread
-      const int row = tid & (kDecSub - 1);
-      const bool isv = tid >= kDecSub;
-      const int key = base + row;
-      int tok = key < n_here ? token_of(key) : -1;
-      const bool ok = tok >= 0;
-      tok = ok ? tok : 0;
-      const float* src = (isv ? p.v_scale : p.k_scale) + (seq0 + tok) * p.Hkv + g;
-      cp_async4(rS + (isv ? kDecSub * 4 : 0) + row * 4, src, ok ? 4u : 0u);
-    }
-  };
   auto load_sub = [&](int st, int stage) {
-    if (FP8) {
-      load_raw(st, stage);
-      return;
-    }
     const uint32_t sK = s_base + stage * kDecStageBytes;
     const uint32_t sV = sK + kDecSub * kKRow;
     const int base = st * kDecSub;
@@ -259,12 +204,6 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
       qa[kk][2] = r0ok ? *reinterpret_cast<const uint32_t*>(qg + gq * kDQK + d0 + 8) : 0u;
       qa[kk][3] = r1ok ? *reinterpret_cast<const uint32_t*>(qg + (gq + 8) * kDQK + d0 + 8) : 0u;
     }
-    if (FP8) {   // S runs as an f16 MMA against the exactly converted K
-#pragma unroll
-      for (int kk = 0; kk < 12; ++kk)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) qa[kk][j] = pack_f16(bf16_lo(qa[kk][j]), bf16_hi(qa[kk][j]));
-    }
   }
 
   float o[16][4];
@@ -272,54 +211,10 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
   for (int j = 0; j < 16; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
 
-  float* s_ks = reinterpret_cast<float*>(smem + kDecStageBytes + 2 * kDecRawBytes);   // FP8
-  float* s_vs = s_ks + kDecSub;
   for (int st = 0; st < nsub; ++st) {
     cp_async_wait<1>();
     __syncthreads();
-    if (FP8) {
-      // raw stage (st & 1) -> converted stage 0: K to f16, V to bf16, scales aside
-      const uint8_t* raw = smem + kDecStageBytes + (st & 1) * kDecRawBytes;
-#pragma unroll
-      for (int i = 0; i < (kDecSub * 12) / kDecThreads; ++i) {
-        const int idx = tid + i * kDecThreads;
-        const int row = idx / 12, u = idx - row * 12;              // 16 bytes -> 2 units
-        const uint4 x = *reinterpret_cast<const uint4*>(raw + row * kKRow8 + u * 16);
-        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-        uint32_t h[8];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          h[2 * j] = e4m3x2_to_f16x2(static_cast<uint16_t>(w[j] & 0xFFFFu));
-          h[2 * j + 1] = e4m3x2_to_f16x2(static_cast<uint16_t>(w[j] >> 16));
-        }
-        const uint32_t dst = s_base + row * kKRow;
-        st_shared_v4(dst + (((2 * u) ^ (row & 7)) << 4), h[0], h[1], h[2], h[3]);
-        st_shared_v4(dst + (((2 * u + 1) ^ (row & 7)) << 4), h[4], h[5], h[6], h[7]);
-      }
-#pragma unroll
-      for (int i = 0; i < (kDecSub * 8) / kDecThreads; ++i) {
-        const int idx = tid + i * kDecThreads;
-        const int row = idx >> 3, u = idx & 7;
-        const uint4 x = *reinterpret_cast<const uint4*>(raw + kDecSub * kKRow8 + row * kVRow8 + u * 16);
-        const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-        uint32_t h[8];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          h[2 * j] = f16x2_to_bf16x2(e4m3x2_to_f16x2(static_cast<uint16_t>(w[j] & 0xFFFFu)));
-          h[2 * j + 1] = f16x2_to_bf16x2(e4m3x2_to_f16x2(static_cast<uint16_t>(w[j] >> 16)));
-        }
-        const uint32_t dst = s_base + kDecSub * kKRow + row * kVRow;
-        st_shared_v4(dst + (((2 * u) ^ (row & 7)) << 4), h[0], h[1], h[2], h[3]);
-        st_shared_v4(dst + (((2 * u + 1) ^ (row & 7)) << 4), h[4], h[5], h[6], h[7]);
-      }
-      s_ks[tid] = reinterpret_cast<const float*>(raw + kDecSub * (kKRow8 + kVRow8))[tid];   // K | V
-      __syncthreads();
-      // raw stage (st & 1) is consumed: refill it now; the converted stage is protected by the
-      // barrier at the top of the next iteration
-      if (st + 2 < nsub) load_sub(st + 2, st & 1);
-      cp_async_commit();
-    }
-    const uint32_t sK = s_base + (FP8 ? 0 : (st & 1) * kDecStageBytes);
+    const uint32_t sK = s_base + (st & 1) * kDecStageBytes;
     const uint32_t sV = sK + kDecSub * kKRow;
     const int mi = lane >> 3, r8 = lane & 7;
 
@@ -333,13 +228,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
         const int unit = 2 * kk + (mi & 1);
         uint32_t b00, b01, b10, b11;
         ldmatrix_x4(rowaddr + ((unit ^ (krow & 7)) << 4), b00, b01, b10, b11);
-        if (FP8) {
-          mma_16816_f16(sacc[0], qa[kk], b00, b01);
-          mma_16816_f16(sacc[1], qa[kk], b10, b11);
-        } else {
-          mma_16816(sacc[0], qa[kk], b00, b01);
-          mma_16816(sacc[1], qa[kk], b10, b11);
-        }
+        mma_16816(sacc[0], qa[kk], b00, b01);
+        mma_16816(sacc[1], qa[kk], b10, b11);
       }
     }
 
@@ -353,8 +243,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
       for (int e = 0; e < 4; ++e) {
         const int key = keybase + nt * 8 + (e & 1);
         const bool ok = key < n_here && (p.mode != kModeSparse || s_tok[key] >= 0);
-        const float ksc = FP8 ? s_ks[keybase - st * kDecSub + nt * 8 + (e & 1)] : 1.f;
-        s[nt][e] = ok ? sacc[nt][e] * ksc * p.scale_log2 : -INFINITY;
+        s[nt][e] = ok ? sacc[nt][e] * p.scale_log2 : -INFINITY;
       }
     }
     float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
@@ -384,15 +273,6 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
       o[j][0] *= al0; o[j][1] *= al0;
       o[j][2] *= al1; o[j][3] *= al1;
     }
-    if (FP8) {   // fold each key's V scale into P (the denominator used the unscaled P)
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        const int kl = keybase - st * kDecSub + nt * 8;
-        const float v0 = s_vs[kl], v1 = s_vs[kl + 1];
-        pv[nt][0] *= v0; pv[nt][1] *= v1;
-        pv[nt][2] *= v0; pv[nt][3] *= v1;
-      }
-    }
     uint32_t pa[4];
     pa[0] = pack_bf16(pv[0][0], pv[0][1]);
     pa[1] = pack_bf16(pv[0][2], pv[0][3]);
@@ -412,11 +292,9 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
         mma_16816(o[2 * jp + 1], pa, v2, v3);
       }
     }
-    if (!FP8) {
-      __syncthreads();
-      if (st + 2 < nsub) load_sub(st + 2, st & 1);
-      cp_async_commit();
-    }
+    __syncthreads();
+    if (st + 2 < nsub) load_sub(st + 2, st & 1);
+    cp_async_commit();
   }
   cp_async_wait<0>();
 
@@ -482,32 +360,69 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
   }
 }
 
-// Merges the chunk states of one (b, h) and adds the sink once:
-// M = max(sink, max_c m_c); L = exp2(sink - M) + sum_c l_c exp2(m_c - M);
-// o = sum_c o_c exp2(m_c - M) / L; lse = (M + log2 L) ln 2.
+// Merges the chunk states of one output row and adds the sink once (one CTA of kDV threads,
+// thread d owning column d): M = max(sink, max_c m_c); L = exp2(sink - M) + sum_c l_c exp2(m_c - M);
+// o = sum_c o_c exp2(m_c - M) / L; lse = (M + log2 L) ln 2. The chunk states are read in
+// parallel (thread t loads chunk t, t + kDV, ...) and the per-column sum runs over weights
+// staged in shared memory, so no thread walks the chunks with a chain of dependent loads.
+// ml: [nvalid][2] (m in log2 units, l), po: [nvalid][kDV]; sk is sink * log2(e) or -inf.
+__device__ __forceinline__ void combine_row(const float* ml, const float* po, int nvalid, float sk,
+                                            bool has_sink, __nv_bfloat16* out_row, float* lse) {
+  __shared__ float s_w[kDV];
+  __shared__ float s_red[kDV / 32];
+  const int d = threadIdx.x, lane = d & 31, warp = d >> 5;
+  float M = sk;
+  for (int c = d; c < nvalid; c += kDV) M = fmaxf(M, ml[2 * c]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  if (lane == 0) s_red[warp] = M;
+  __syncthreads();
+#pragma unroll
+  for (int w = 0; w < kDV / 32; ++w) M = fmaxf(M, s_red[w]);
+  const float ref = M == -INFINITY ? 0.f : M;
+  float lpart = 0.f, acc = 0.f;
+  for (int c0 = 0; c0 < nvalid; c0 += kDV) {
+    const int c = c0 + d;
+    float w = 0.f;
+    if (c < nvalid) {
+      w = ex2(ml[2 * c] - ref);
+      lpart += ml[2 * c + 1] * w;
+    }
+    __syncthreads();                 // the previous tile's weights (and s_red) are consumed
+    s_w[d] = w;
+    __syncthreads();
+    const int n = nvalid - c0 < kDV ? nvalid - c0 : kDV;
+    const float* pc = po + static_cast<long long>(c0) * kDV + d;
+#pragma unroll 8
+    for (int i = 0; i < n; ++i) acc += pc[i * kDV] * s_w[i];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) lpart += __shfl_xor_sync(0xffffffffu, lpart, o);
+  __syncthreads();
+  if (lane == 0) s_red[warp] = lpart;
+  __syncthreads();
+  float Lt = has_sink ? ex2(sk - ref) : 0.f;
+#pragma unroll
+  for (int w = 0; w < kDV / 32; ++w) Lt += s_red[w];
+  const float ov = Lt > 0.f ? acc / Lt : 0.f;
+  out_row[d] = __float2bfloat16_rn(ov);
+  if (d == 0 && lse) *lse = Lt > 0.f ? (ref + log2f(Lt)) * 0.6931471805599453f : -INFINITY;
+}
+
+// Merges the chunk states of one (b, h) of a decode call (combine_row).
 __global__ void __launch_bounds__(kDV) decode_combine_kernel(const DecodeParams p) {
+  pdl_wait();
+  pdl_trigger();
   const int bh = blockIdx.x;
   const int b = bh / p.Hq, h = bh - b * p.Hq;
-  const int d = threadIdx.x;
   int nw, L;
   const int nkeys = dec_unit_keys(p, b, nw, L);
   int nvalid = (nkeys + p.chunk - 1) / p.chunk;
   nvalid = nvalid < p.nchunks ? nvalid : p.nchunks;
   const float sk = p.sink ? p.sink[h] * 1.4426950408889634f : -INFINITY;
-  const float* ml = p.part_ml + static_cast<long long>(bh) * p.nchunks * 2;
-  const float* po = p.part_o + static_cast<long long>(bh) * p.nchunks * kDV;
-  float M = sk;
-  for (int c = 0; c < nvalid; ++c) M = fmaxf(M, ml[2 * c]);
-  const float ref = M == -INFINITY ? 0.f : M;
-  float Lt = p.sink ? ex2(sk - ref) : 0.f, acc = 0.f;
-  for (int c = 0; c < nvalid; ++c) {
-    const float sc = ex2(ml[2 * c] - ref);
-    Lt += ml[2 * c + 1] * sc;
-    acc += po[c * kDV + d] * sc;
-  }
-  const float ov = Lt > 0.f ? acc / Lt : 0.f;
-  p.out[static_cast<long long>(bh) * kDV + d] = __float2bfloat16_rn(ov);
-  if (d == 0 && p.lse) p.lse[bh] = Lt > 0.f ? (ref + log2f(Lt)) * 0.6931471805599453f : -INFINITY;
+  combine_row(p.part_ml + static_cast<long long>(bh) * p.nchunks * 2,
+              p.part_o + static_cast<long long>(bh) * p.nchunks * kDV, nvalid, sk, p.sink != nullptr,
+              p.out + static_cast<long long>(bh) * kDV, p.lse ? p.lse + bh : nullptr);
 }
 
 // Debug check of sparse preconditions; one thread per (b, g) row. A valid row is a strictly

@@ -60,6 +60,8 @@ __device__ __forceinline__ int mq_range(const DecodeMqParams& p, int b, int& klo
 template <int G>
 __global__ void __launch_bounds__(kDecThreads, 2) decode_mq_kernel(const DecodeMqParams p) {
   static_assert(G >= 1 && G <= 16, "group size");
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(1024) uint8_t smem[];
   const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -286,33 +288,22 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_mq_kernel(const DecodeM
   }
 }
 
-// Merges the chunk states of one (b, t, h) row and adds the sink once (as
-// decode_combine_kernel, over the chunks that hold keys of the unit).
+// Merges the chunk states of one (b, t, h) row and adds the sink once (combine_row, over the
+// chunks that hold keys of the unit).
 __global__ void __launch_bounds__(kDV) decode_mq_combine_kernel(const DecodeMqParams p) {
+  pdl_wait();
+  pdl_trigger();
   const long long row = blockIdx.x;
   const int h = static_cast<int>(row % p.Hq);
   const int b = static_cast<int>(row / (static_cast<long long>(p.T) * p.Hq));
-  const int d = threadIdx.x;
   int klo;
   const int L = mq_range(p, b, klo);
   const int nkeys = L - klo > 0 ? L - klo : 0;
   int nvalid = (nkeys + p.chunk - 1) / p.chunk;
   nvalid = nvalid < p.nchunks ? nvalid : p.nchunks;
   const float sk = p.sink ? p.sink[h] * 1.4426950408889634f : -INFINITY;
-  const float* ml = p.part_ml + row * p.nchunks * 2;
-  const float* po = p.part_o + row * p.nchunks * kDV;
-  float M = sk;
-  for (int cc = 0; cc < nvalid; ++cc) M = fmaxf(M, ml[2 * cc]);
-  const float ref = M == -INFINITY ? 0.f : M;
-  float Lt = p.sink ? ex2(sk - ref) : 0.f, acc = 0.f;
-  for (int cc = 0; cc < nvalid; ++cc) {
-    const float sc = ex2(ml[2 * cc] - ref);
-    Lt += ml[2 * cc + 1] * sc;
-    acc += po[cc * kDV + d] * sc;
-  }
-  const float ov = Lt > 0.f ? acc / Lt : 0.f;
-  p.out[row * kDV + d] = __float2bfloat16_rn(ov);
-  if (d == 0 && p.lse) p.lse[row] = Lt > 0.f ? (ref + log2f(Lt)) * 0.6931471805599453f : -INFINITY;
+  combine_row(p.part_ml + row * p.nchunks * 2, p.part_o + row * p.nchunks * kDV, nvalid, sk, p.sink != nullptr,
+              p.out + row * kDV, p.lse ? p.lse + row : nullptr);
 }
 
 }  // namespace mimo

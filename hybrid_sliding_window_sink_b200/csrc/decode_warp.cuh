@@ -161,6 +161,8 @@ template <int G, int NS>
 __global__ void __launch_bounds__(32) decode_warp_kernel(const DecodeParams p) {
   static_assert(G >= 1 && G <= 16, "group size");
   static_assert(NS >= 1 && NS <= kDwMaxStages, "stages in flight");
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ __align__(1024) uint8_t smem[];
   const int c = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int lane = threadIdx.x, gq = lane >> 2, tq = lane & 3;

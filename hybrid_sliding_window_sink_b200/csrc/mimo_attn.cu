@@ -16,13 +16,13 @@
 #include "decode.cuh"
 #include "decode_mq.cuh"
 #include "decode_warp.cuh"
+#include "decode_fp8.cuh"
 #include "select.cuh"
 #include "prefill.cuh"
 #include "prefill_swa.cuh"
 #include "prefill_ga.cuh"
 
 namespace mimo {
-__device__ unsigned g_device_error = 0;
 
 #ifdef MIMO_TEST_HOOKS
 // Test builds only: one warp waits on an mbarrier that nothing ever arrives on, through the
@@ -301,6 +301,28 @@ mimo_status prefill_chunk_group(const mimo_shape* s, const void* q, const void* 
   return launch_prefill<G, 128, 2>(s, q, k, v, prm, sms, st);
 }
 
+// Launches a decode-side kernel, with programmatic stream serialization when `pdl` is set: its
+// CTAs may then be scheduled while the previous kernel on the stream drains (each kernel's
+// first statement is pdl_wait, so nothing is read before that kernel has completed). Used for
+// the combine that follows a split-KV kernel; the one-kernel SWA ring layers of the decode step
+// measured slower launched this way (14.9 -> 16.8-17.3 us per layer), so the split kernels are
+// launched plainly (their pdl_wait is then a no-op).
+template <typename P>
+cudaError_t launch_pdl(void (*kern)(P), dim3 grid, int threads, size_t smem, cudaStream_t st, const P& prm,
+                       bool pdl = true) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(static_cast<unsigned>(threads));
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, prm);
+}
+
 // ---------------------------------------------------------------- decode
 struct DecodePlan {
   int chunk, nchunks, direct;
@@ -373,6 +395,64 @@ DecodePlan plan_decode_warp(const mimo_shape* s, int mode, int cap, int recent, 
   return pl;
 }
 
+// Plan of the FP8 decode calls (decode_fp8_kernel, one warp per CTA): a sparse unit in chunks
+// of 64 keys (two stages, both in flight); a ring unit of at most 256 keys in one chunk,
+// finalised in place, with four stages of 32 keys in flight; a longer (linear) unit in chunks
+// of 256 .. 2048 keys, about 32 CTAs per SM in all so that uneven lengths balance, with two
+// stages in flight: 21 KB of shared memory per CTA, so that registers (eight warps per SM)
+// rather than shared memory bound the warps an SM holds (measured: 0.65 of HBM against 0.55
+// with four stages and 0.63 with three on the 9 GA layers of the FP8 decode step).
+DecodePlan plan_decode_fp8(const mimo_shape* s, int mode, int cap, int recent, int n_sel, int sms,
+                           int* stages) {
+  long long total = mode == mimo::kModeSparse ? static_cast<long long>(recent) + n_sel : cap;
+  if (total < 1) total = 1;
+  const long long units = static_cast<long long>(s->batch) * s->n_kv_heads;
+  DecodePlan pl{};
+  if (mode == mimo::kModeSparse) {
+    *stages = 2;
+    pl.chunk = 64;
+  } else if (total <= 256) {
+    *stages = 4;
+    pl.chunk = static_cast<int>((total + 31) / 32 * 32);
+  } else {
+    *stages = 2;
+    const int ch = pow2_floor(total * units / (32LL * sms));
+    pl.chunk = ch < 256 ? 256 : (ch > 2048 ? 2048 : ch);
+  }
+  if (pl.chunk > total) pl.chunk = static_cast<int>((total + 31) / 32 * 32);
+  pl.nchunks = static_cast<int>((total + pl.chunk - 1) / pl.chunk);
+  pl.direct = pl.nchunks == 1;
+  if (pl.direct) {
+    pl.bytes = 0;
+  } else {
+    const size_t rows = static_cast<size_t>(s->batch) * s->n_q_heads * pl.nchunks;
+    const size_t ml = (rows * 2 * sizeof(float) + 255) / 256 * 256;
+    pl.bytes = ml + rows * mimo::kDV * sizeof(float);
+  }
+  return pl;
+}
+
+template <int G, int NS>
+mimo_status launch_decode_fp8_g(DecodeParams prm, cudaStream_t st) {
+  auto kern = mimo::decode_fp8_kernel<G, NS>;
+  const int smem = mimo::d8_smem_bytes(NS);
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
+    cudaGetLastError();
+    return MIMO_ERR_CUDA;
+  }
+  dim3 grid(prm.nchunks, prm.Hkv, prm.B);
+  if (launch_pdl(kern, grid, 32, smem, st, prm, false) != cudaSuccess) return MIMO_ERR_CUDA;
+  if (!prm.direct &&
+      launch_pdl(mimo::decode_combine_kernel, dim3(prm.B * prm.Hq), mimo::kDV, 0, st, prm) != cudaSuccess)
+    return MIMO_ERR_CUDA;
+  return MIMO_OK;
+}
+
+template <int G>
+mimo_status launch_decode_fp8_gs(DecodeParams prm, cudaStream_t st) {
+  return prm.nstages == 2 ? launch_decode_fp8_g<G, 2>(prm, st) : launch_decode_fp8_g<G, 4>(prm, st);
+}
+
 template <int G>
 mimo_status launch_decode_warp_g(DecodeParams prm, cudaStream_t st) {
   auto kern = mimo::decode_warp_kernel<G, 2>;
@@ -382,30 +462,26 @@ mimo_status launch_decode_warp_g(DecodeParams prm, cudaStream_t st) {
     return MIMO_ERR_CUDA;
   }
   dim3 grid(prm.nchunks, prm.Hkv, prm.B);
-  kern<<<grid, 32, smem, st>>>(prm);
-  if (cudaGetLastError() != cudaSuccess) return MIMO_ERR_CUDA;
-  if (!prm.direct) {
-    mimo::decode_combine_kernel<<<prm.B * prm.Hq, mimo::kDV, 0, st>>>(prm);
-    if (cudaGetLastError() != cudaSuccess) return MIMO_ERR_CUDA;
-  }
+  if (launch_pdl(kern, grid, 32, smem, st, prm, false) != cudaSuccess) return MIMO_ERR_CUDA;
+  if (!prm.direct &&
+      launch_pdl(mimo::decode_combine_kernel, dim3(prm.B * prm.Hq), mimo::kDV, 0, st, prm) != cudaSuccess)
+    return MIMO_ERR_CUDA;
   return MIMO_OK;
 }
 
-template <int G, bool FP8 = false>
+template <int G>
 mimo_status launch_decode_g(DecodeParams prm, cudaStream_t st) {
-  auto kern = mimo::decode_split_kernel<G, FP8>;
-  const int smem = FP8 ? mimo::kDecSmemBytesFp8 : mimo::kDecSmemBytes;
+  auto kern = mimo::decode_split_kernel<G>;
+  const int smem = mimo::kDecSmemBytes;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
     cudaGetLastError();
     return MIMO_ERR_CUDA;
   }
   dim3 grid(prm.nchunks, prm.Hkv, prm.B);
-  kern<<<grid, mimo::kDecThreads, smem, st>>>(prm);
-  if (cudaGetLastError() != cudaSuccess) return MIMO_ERR_CUDA;
-  if (!prm.direct) {
-    mimo::decode_combine_kernel<<<prm.B * prm.Hq, mimo::kDV, 0, st>>>(prm);
-    if (cudaGetLastError() != cudaSuccess) return MIMO_ERR_CUDA;
-  }
+  if (launch_pdl(kern, grid, mimo::kDecThreads, smem, st, prm, false) != cudaSuccess) return MIMO_ERR_CUDA;
+  if (!prm.direct &&
+      launch_pdl(mimo::decode_combine_kernel, dim3(prm.B * prm.Hq), mimo::kDV, 0, st, prm) != cudaSuccess)
+    return MIMO_ERR_CUDA;
   return MIMO_OK;
 }
 
@@ -431,7 +507,7 @@ mimo_status run_decode(const mimo_shape* s, int mode, const void* q, const void*
   if (dev < 0) return MIMO_ERR_CUDA;
   const int sms = sm_count_for(dev);
   int stages = 2;
-  const DecodePlan pl = fp8 ? plan_decode(s, mode, cap, recent, n_sel, sms)
+  const DecodePlan pl = fp8 ? plan_decode_fp8(s, mode, cap, recent, n_sel, sms, &stages)
                             : plan_decode_warp(s, mode, cap, recent, n_sel, sms, &stages);
   if (pl.bytes > 0 && (!ws || ws_bytes < pl.bytes)) return MIMO_ERR_WORKSPACE;
   if (ws && !aligned(ws, 16)) return MIMO_ERR_ALIGN;
@@ -486,11 +562,11 @@ mimo_status run_decode(const mimo_shape* s, int mode, const void* q, const void*
   }
   if (fp8) {
     switch (prm.group) {
-      case 1: return launch_decode_g<1, true>(prm, st);
-      case 2: return launch_decode_g<2, true>(prm, st);
-      case 4: return launch_decode_g<4, true>(prm, st);
-      case 8: return launch_decode_g<8, true>(prm, st);
-      default: return launch_decode_g<16, true>(prm, st);
+      case 1: return launch_decode_fp8_gs<1>(prm, st);
+      case 2: return launch_decode_fp8_gs<2>(prm, st);
+      case 4: return launch_decode_fp8_gs<4>(prm, st);
+      case 8: return launch_decode_fp8_gs<8>(prm, st);
+      default: return launch_decode_fp8_gs<16>(prm, st);
     }
   }
   switch (prm.group) {
@@ -544,13 +620,14 @@ mimo_status launch_decode_mq_g(const mimo::DecodeMqParams& prm, cudaStream_t st)
     return MIMO_ERR_CUDA;
   }
   dim3 grid(prm.nchunks, prm.Hkv, prm.B);
-  kern<<<grid, mimo::kDecThreads, mimo::kDecSmemBytes, st>>>(prm);
-  if (cudaGetLastError() != cudaSuccess) return MIMO_ERR_CUDA;
+  if (launch_pdl(kern, grid, mimo::kDecThreads, mimo::kDecSmemBytes, st, prm, false) != cudaSuccess)
+    return MIMO_ERR_CUDA;
   if (!prm.direct) {
     const long long rows = static_cast<long long>(prm.B) * prm.T * prm.Hq;
     if (rows > 0x7fffffffLL) return MIMO_ERR_UNSUPPORTED;
-    mimo::decode_mq_combine_kernel<<<static_cast<unsigned>(rows), mimo::kDV, 0, st>>>(prm);
-    if (cudaGetLastError() != cudaSuccess) return MIMO_ERR_CUDA;
+    if (launch_pdl(mimo::decode_mq_combine_kernel, dim3(static_cast<unsigned>(rows)), mimo::kDV, 0, st, prm) !=
+        cudaSuccess)
+      return MIMO_ERR_CUDA;
   }
   return MIMO_OK;
 }
@@ -883,11 +960,11 @@ size_t mimo_attn_workspace_size(const mimo_shape* s, int op, int cache_kind, int
   } else {
     return 0;
   }
-  // one size serves both the bf16 calls (one-warp kernel plan) and the FP8 calls
+  // one size serves both the bf16 calls and the FP8 calls
   const int sms = sm_count_for(current_device());
   int stages = 2;
   return std::max(plan_decode_warp(s, mode, cache_capacity, recent, n_sel, sms, &stages).bytes,
-                  plan_decode(s, mode, cache_capacity, recent, n_sel, sms).bytes);
+                  plan_decode_fp8(s, mode, cache_capacity, recent, n_sel, sms, &stages).bytes);
 }
 
 mimo_status mimo_attn_check_indices(const mimo_shape* s, const int* lengths, const int* sel_idx,

@@ -11,15 +11,21 @@
 namespace mimo {
 
 // ---------------------------------------------------------------------------
-// Device error word. Kernels OR a code into it when a bounded wait gives up;
-// the host reads and clears it with mimo_attn_last_device_error().
+// Device error word. Kernels OR a code into it when a bounded wait gives up (and, in debug
+// builds, when an input is out of range); the host reads and clears it with
+// mimo_attn_last_device_error().
 // ---------------------------------------------------------------------------
 enum : unsigned {
   kErrWaitTimeout = 1u,   // an mbarrier wait exceeded its time limit
   kErrDrainTimeout = 2u,  // waiting for in-flight copies / MMAs at exit gave up
   kErrBadLength = 4u,     // (debug builds) a sequence length outside [0, capacity]
   kErrBadIndex = 8u,      // (debug builds) a selected index outside [0, L - recent), or unsorted
+  kErrF16Range = 16u,     // (debug builds) an operand carried in f16 was beyond +-65504 or NaN
 };
+
+// The word itself. The library is one translation unit (mimo_attn.cu includes every kernel
+// header once), so the definition lives here, next to the codes.
+__device__ unsigned g_device_error = 0;
 
 // Wall-clock limit for a wait on work in progress (nanoseconds): 2 s. A test build sets
 // MIMO_WAIT_LIMIT_NS to a few nanoseconds so that waits give up and the abort path runs.
@@ -40,6 +46,17 @@ __device__ __forceinline__ unsigned long long globaltimer_ns() {
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
+
+// ---------------------------------------------------------------------------
+// Programmatic dependent launch. A kernel launched with programmatic stream serialization may
+// be scheduled while the kernel before it on the stream drains. pdl_wait blocks until that
+// kernel has completed and its writes are visible (a no-op for a kernel launched without the
+// attribute), so it precedes every global-memory access of the kernel; pdl_trigger lets the
+// next such kernel be scheduled once every CTA of this one has started (that kernel still
+// waits for this one to complete before it reads anything).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------
 // mbarrier
@@ -269,13 +286,22 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }
+// Debug builds record (and still convert) any value that the f16 carrying would change by
+// more than rounding: beyond the finite f16 range, or NaN. Product builds compile it away.
+__device__ __forceinline__ void check_f16_range(float lo, float hi) {
+#ifdef MIMO_DEBUG
+  if (!(fabsf(lo) <= 65504.f) || !(fabsf(hi) <= 65504.f)) atomicOr(&g_device_error, kErrF16Range);
+#endif
+}
 // Round to f16 with values beyond the f16 range clamped to +-65504 (one cvt with satfinite).
 __device__ __forceinline__ uint32_t pack_f16_sat(float lo, float hi) {
+  check_f16_range(lo, hi);
   uint32_t r;
   asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
 __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  check_f16_range(lo, hi);
   __half2 v = __floats2half2_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
 }

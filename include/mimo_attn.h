@@ -34,8 +34,11 @@
  *    query head h reads KV head h / group (contiguous groups).
  *  - Precision: products of bf16 inputs are exact and accumulate in fp32. The RoPE-rotated
  *    Q/K dims (prefill) are carried in f16 for their MMAs, and the SWA prefill kernel keeps
- *    P and V in f16; inputs are therefore expected inside the f16 range (|x| < 65504) -
- *    values outside it are clamped. Outputs are rounded to bf16, lse is fp32.
+ *    P and V in f16; inputs are therefore expected inside the f16 range (|x| <= 65504, and
+ *    a rotated pair's norm too) - values outside it are clamped. The FP8 decode converts Q
+ *    to f16 without clamping (a larger |q| becomes infinite). A build compiled with
+ *    MIMO_DEBUG records every such value in the device error word (bit 16, see
+ *    mimo_attn_last_device_error). Outputs are rounded to bf16, lse is fp32.
  *  - Thread safety: calls may be made from several host threads; the shared mutable
  *    state is the device error word read by mimo_attn_last_device_error and the scratch
  *    array of mimo_attn_sparse_noalloc (see there).
@@ -253,9 +256,10 @@ size_t mimo_attn_decode_mq_workspace_size(const mimo_shape* shape, int cache_kin
  *  kind and sizes) and the errors: as mimo_attn_decode / mimo_attn_sparse; MIMO_ERR_NULL
  *  also for a missing scale array.
  *
- * The E4M3 bytes are converted exactly (K to f16, V to bf16); the K scale multiplies the
- * fp32 score and the V scale multiplies P before its bf16 rounding. q must lie inside the
- * f16 range (|q| < 65504) because S = Q K^T runs as an f16 MMA.
+ * The E4M3 bytes are converted exactly to f16 (K and V); the K scale multiplies the fp32
+ * score and the V scale multiplies P, which is rounded to f16 after a power-of-two factor per
+ * 32 keys that keeps it below 2 (the factor is divided out of the output). q must lie inside
+ * the f16 range (|q| <= 65504) because S = Q K^T runs as an f16 MMA.
  */
 mimo_status mimo_attn_decode_fp8(const mimo_shape* shape, const void* q, const void* k_cache,
                                  const void* v_cache, const float* k_scale, const float* v_scale,
@@ -350,9 +354,11 @@ mimo_status mimo_attn_check_indices(const mimo_shape* shape, const int* lengths,
  * gave up (2 s; the kernel then left its loops, waited for its own copies and MMAs in flight,
  * freed its tensor memory and returned without finishing its output), 2 = one of those
  * exit-path waits gave up too, and in builds compiled with MIMO_DEBUG 4 = a sequence length
- * outside [0, capacity] and 8 = a selected index outside [0, L - recent) or not increasing
- * (both clamped, so no access leaves the caller's buffers). Host-blocking; for tests and
- * debugging. Returns 0xFFFFFFFF if the device could not be synchronised. */
+ * outside [0, capacity], 8 = a selected index outside [0, L - recent) or not increasing
+ * (both clamped, so no access leaves the caller's buffers) and 16 = an operand carried in
+ * f16 (see Precision) beyond +-65504 or NaN (converted as in the product build).
+ * Host-blocking; for tests and debugging. Returns 0xFFFFFFFF if the device could not be
+ * synchronised. */
 unsigned int mimo_attn_last_device_error(void);
 
 /* mimo_attn_last_device_error as a status: MIMO_OK when the word was 0, MIMO_ERR_DEVICE

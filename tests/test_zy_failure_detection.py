@@ -8,7 +8,8 @@ ORs a bit into the device error word and returns. Two test builds of the same so
 * shortwait: waits on work in progress give up after 1 ns, so the abort paths of the real
   kernels run; it also has a hook that waits on a barrier nothing ever arrives on.
 * debug: kernels record lengths and selected indices outside their ranges in the error word
-  (and still clamp them, so no access leaves the caller's buffers).
+  (and still clamp them, so no access leaves the caller's buffers), and every operand they
+  carry in f16 that lies beyond +-65504.
 
 After each, the product build runs on the same CUDA context and must give correct results.
 """
@@ -27,7 +28,7 @@ from parity_util import compare
 pytestmark = pytest.mark.gpu
 
 MIMO_OK, MIMO_ERR_DEVICE = 0, 7
-WAIT_TIMEOUT, DRAIN_TIMEOUT, BAD_LENGTH, BAD_INDEX = 1, 2, 4, 8
+WAIT_TIMEOUT, DRAIN_TIMEOUT, BAD_LENGTH, BAD_INDEX, F16_RANGE = 1, 2, 4, 8, 16
 
 
 @contextlib.contextmanager
@@ -137,3 +138,68 @@ def test_debug_build_reports_bad_lengths_and_indices(cuda_device):
         o_ref, l_ref = ref.decode(wl.to_f64(d["q"]), wl.to_f64(d["k_cache"]), wl.to_f64(d["v_cache"]), "linear",
                                   [cap, 10], wl.to_f64(d["sink"]))
         compare(wl.to_f64(out), o_ref, wl.to_f64(lse), l_ref, "debug build, clamped length")
+
+
+def _bf16(x, s):
+    return (x.float() * s).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("n, hq, hkv, window, theta", [
+    (640, 64, 8, 128, 1e4),      # SWA ring kernel: rotated Q/K, P and V in f16
+    (384, 64, 4, 0, 1e7),        # GA pair kernel: rotated Q/K in f16
+    (300, 16, 4, 64, 1e4),       # generic kernel: rotated Q/K in f16
+])
+def test_debug_build_reports_operands_beyond_the_f16_range(cuda_device, n, hq, hkv, window, theta):
+    """In the debug build, K and V in the thousands (inside the f16 range) leave the word clear
+    and match the oracle; one K entry of 1e5 in a rotated dim sets the f16-range bit, the same
+    entry in a dim carried in bf16 does not; a V entry of 1e5 sets it in the SWA ring kernel,
+    the one kernel that carries V in f16."""
+    dev = cuda_device
+    x = wl.prefill_inputs(1, n, hq, hkv, seed=66 + n)
+    q, k, v = _bf16(x["q"], 1e-3), _bf16(x["k"], 1e3), _bf16(x["v"], 2e3)
+    sink = x["sink"].to(dev)
+
+    def run(kk, vv):
+        out, lse = _lib.prefill(q.to(dev), kk.to(dev), vv.to(dev), sink, window=window,
+                                rope_theta=theta, rot_dims=64)
+        torch.cuda.synchronize()
+        return out, lse
+
+    with _library("debug") as lib:
+        out, lse = run(k, v)
+        assert _status(lib) == (MIMO_OK, 0)
+        o_ref, l_ref = ref.prefill(wl.to_f64(q), wl.to_f64(k), wl.to_f64(v), wl.to_f64(x["sink"]), window,
+                                   theta, 64)
+        compare(wl.to_f64(out) / 2e3, o_ref / 2e3, wl.to_f64(lse), l_ref, f"debug build, W={window}")
+        k_rot = k.clone()
+        k_rot[0, n // 2, 0, 5] = 1e5             # dims 0..63 are rotated
+        run(k_rot, v)
+        assert _status(lib) == (MIMO_ERR_DEVICE, F16_RANGE)
+        k_plain = k.clone()
+        k_plain[0, n // 2, 0, 150] = 1e5         # an unrotated dim, multiplied in bf16
+        out, _ = run(k_plain, v)
+        assert _status(lib) == (MIMO_OK, 0)
+        assert torch.isfinite(out).all()
+        v_big = v.clone()
+        v_big[0, n // 2, 0, 9] = 1e5
+        run(k, v_big)
+        assert _status(lib) == ((MIMO_ERR_DEVICE, F16_RANGE) if (window, hkv) == (128, 8) else (MIMO_OK, 0))
+
+
+def test_debug_build_reports_an_fp8_decode_query_beyond_the_f16_range(cuda_device):
+    """The FP8 decode multiplies Q in f16: a query entry of 1e5 sets the f16-range bit in the
+    debug build; the same call with the query in range leaves it clear."""
+    dev = cuda_device
+    lengths = [700, 4096]
+    inp = wl.decode_fp8_inputs(2, 64, 4, 4096, lengths, seed=69)
+    d = {k: v.to(dev) for k, v in inp.items() if v is not None}
+    with _library("debug") as lib:
+        _lib.decode_fp8(d["q"], d["k8"], d["v8"], d["k_scale"], d["v_scale"], d["lengths"], d["sink"],
+                        kind="linear")
+        torch.cuda.synchronize()
+        assert _status(lib) == (MIMO_OK, 0)
+        q = d["q"].clone()
+        q[1, 3, 17] = 1e5
+        _lib.decode_fp8(q, d["k8"], d["v8"], d["k_scale"], d["v_scale"], d["lengths"], d["sink"], kind="linear")
+        torch.cuda.synchronize()
+        assert _status(lib) == (MIMO_ERR_DEVICE, F16_RANGE)
