@@ -304,9 +304,11 @@ mimo_status prefill_chunk_group(const mimo_shape* s, const void* q, const void* 
 // Launches a decode-side kernel, with programmatic stream serialization when `pdl` is set: its
 // CTAs may then be scheduled while the previous kernel on the stream drains (each kernel's
 // first statement is pdl_wait, so nothing is read before that kernel has completed). Used for
-// the combine that follows a split-KV kernel; the one-kernel SWA ring layers of the decode step
-// measured slower launched this way (14.9 -> 16.8-17.3 us per layer), so the split kernels are
-// launched plainly (their pdl_wait is then a no-op).
+// the combine that follows a split-KV kernel and for the one-warp split kernels when a combine
+// follows them (sparse call: 15.0 -> 14.5 us with the combine alone, 14.1 us with both); the
+// one-kernel SWA ring layers measured slower launched this way (14.9 -> 16.8-17.3 us per layer)
+// and the four-warp GA kernels no faster, so those are launched plainly (pdl_wait is then a
+// no-op).
 template <typename P>
 cudaError_t launch_pdl(void (*kern)(P), dim3 grid, int threads, size_t smem, cudaStream_t st, const P& prm,
                        bool pdl = true) {
@@ -441,7 +443,7 @@ mimo_status launch_decode_fp8_g(DecodeParams prm, cudaStream_t st) {
     return MIMO_ERR_CUDA;
   }
   dim3 grid(prm.nchunks, prm.Hkv, prm.B);
-  if (launch_pdl(kern, grid, 32, smem, st, prm, false) != cudaSuccess) return MIMO_ERR_CUDA;
+  if (launch_pdl(kern, grid, 32, smem, st, prm, !prm.direct) != cudaSuccess) return MIMO_ERR_CUDA;
   if (!prm.direct &&
       launch_pdl(mimo::decode_combine_kernel, dim3(prm.B * prm.Hq), mimo::kDV, 0, st, prm) != cudaSuccess)
     return MIMO_ERR_CUDA;
@@ -462,7 +464,7 @@ mimo_status launch_decode_warp_g(DecodeParams prm, cudaStream_t st) {
     return MIMO_ERR_CUDA;
   }
   dim3 grid(prm.nchunks, prm.Hkv, prm.B);
-  if (launch_pdl(kern, grid, 32, smem, st, prm, false) != cudaSuccess) return MIMO_ERR_CUDA;
+  if (launch_pdl(kern, grid, 32, smem, st, prm, !prm.direct) != cudaSuccess) return MIMO_ERR_CUDA;
   if (!prm.direct &&
       launch_pdl(mimo::decode_combine_kernel, dim3(prm.B * prm.Hq), mimo::kDV, 0, st, prm) != cudaSuccess)
     return MIMO_ERR_CUDA;
