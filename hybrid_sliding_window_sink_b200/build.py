@@ -20,7 +20,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB_NAME = "libmimo_attn.so"
 LIB_PATH = os.path.join(PKG, LIB_NAME)
 SOURCES = ["mimo_attn.cu"]
-HEADERS = ["ptx.cuh", "decode.cuh", "decode_warp.cuh", "decode_fp8.cuh", "decode_mq.cuh", "select.cuh", "prefill.cuh", "prefill_swa.cuh", "prefill_ga.cuh"]
+HEADERS = ["ptx.cuh", "decode.cuh", "decode_warp.cuh", "decode_fp8.cuh", "decode_mq_tma.cuh", "decode_mq.cuh", "select.cuh", "prefill.cuh", "prefill_swa.cuh", "prefill_ga.cuh"]
 
 
 def nvcc_path() -> str:

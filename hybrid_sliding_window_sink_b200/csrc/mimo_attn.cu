@@ -17,6 +17,7 @@
 #include "decode_mq.cuh"
 #include "decode_warp.cuh"
 #include "decode_fp8.cuh"
+#include "decode_mq_tma.cuh"
 #include "select.cuh"
 #include "prefill.cuh"
 #include "prefill_swa.cuh"
@@ -613,8 +614,37 @@ mimo_status check_mq(const mimo_shape* s, int cache_kind, int cap, int T, int W)
   return MIMO_OK;
 }
 
+// Multi-query decode over a linear (GA) cache: decode_mq_tma_kernel (TMA-fed K/V subtiles,
+// S and PV on tcgen05, O in TMEM, one CTA per SM). Ring caches, whose subtiles wrap around the
+// ring, stay on decode_mq_kernel (cp.async gathers, mma.sync).
+template <int G>
+mimo_status launch_decode_mq_tma_g(const mimo::DecodeMqParams& prm, cudaStream_t st) {
+  CUtensorMap tk, tv;
+  if (!make_tmap(&tk, prm.k, mimo::kDQK, prm.Hkv, prm.seq_stride, prm.B, 1, mimo::kMtKeys) ||
+      !make_tmap(&tv, prm.v, mimo::kDV, prm.Hkv, prm.seq_stride, prm.B, 1, mimo::kMtKeys))
+    return MIMO_ERR_CUDA;
+  auto kern = mimo::decode_mq_tma_kernel<G>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, mimo::kMtSmemBytes) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return MIMO_ERR_CUDA;
+  }
+  dim3 grid(prm.nchunks, prm.Hkv, prm.B);
+  kern<<<grid, mimo::kMtThreads, mimo::kMtSmemBytes, st>>>(tk, tv, prm);
+  if (cudaGetLastError() != cudaSuccess) return MIMO_ERR_CUDA;
+  if (!prm.direct) {
+    const long long rows = static_cast<long long>(prm.B) * prm.T * prm.Hq;
+    if (rows > 0x7fffffffLL) return MIMO_ERR_UNSUPPORTED;
+    if (launch_pdl(mimo::decode_mq_combine_kernel, dim3(static_cast<unsigned>(rows)), mimo::kDV, 0, st, prm) !=
+        cudaSuccess)
+      return MIMO_ERR_CUDA;
+  }
+  return MIMO_OK;
+}
+
 template <int G>
 mimo_status launch_decode_mq_g(const mimo::DecodeMqParams& prm, cudaStream_t st) {
+  if (prm.mode == mimo::kModeLinear) return launch_decode_mq_tma_g<G>(prm, st);
   auto kern = mimo::decode_mq_kernel<G>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, mimo::kDecSmemBytes) !=
       cudaSuccess) {
