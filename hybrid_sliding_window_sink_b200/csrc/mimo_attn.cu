@@ -866,7 +866,7 @@ mimo_status mimo_attn_select_tokens(const mimo_shape* s, const void* q, const vo
   }
   if (!launched) return MIMO_ERR_CUDA;
   if (cudaGetLastError() != cudaSuccess) return MIMO_ERR_CUDA;
-  mimo::select_topk_kernel<<<dim3(s->n_kv_heads, s->batch), mimo::kSelThreads, 0, st>>>(prm);
+  mimo::select_topk_kernel<<<dim3(s->n_kv_heads * mimo::kSelCluster, s->batch), mimo::kSelThreads, 0, st>>>(prm);
   return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ERR_CUDA;
 }
 

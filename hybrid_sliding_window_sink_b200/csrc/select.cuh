@@ -27,6 +27,7 @@ constexpr int kSelThreads = 1024;
 constexpr int kSelPerThread = 16;                 // candidates per thread per compaction step
 constexpr int kSelBlockKeys = kSelPerThread * kSelThreads;
 constexpr int kSelUnroll = 8;                     // 16-byte key loads in flight per thread
+constexpr int kSelCluster = 8;                    // CTAs per (b, g) in the top-k
 
 struct SelectParams {
   const __nv_bfloat16* q;     // [B, Hq, 192]
@@ -219,12 +220,41 @@ __device__ __forceinline__ void select_pick_bin(const int* s_hist, int shift, ui
   }
 }
 
-__global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const SelectParams p) {
-  __shared__ int s_hist[256];
+// Cluster helpers: the shared-memory address of `saddr` in CTA `rank` of this cluster, a
+// 32-bit load from it, and a cluster-wide barrier (release / acquire).
+__device__ __forceinline__ uint32_t cluster_map(uint32_t saddr, int rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ int ld_cluster_s32(uint32_t addr) {
+  int v;
+  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
+}
+
+// Top-k per (b, g) on a cluster of kSelCluster CTAs: CTA `rank` owns the contiguous candidate
+// slice [lo, hi_c). Digit 1 of the radix select is summed from the score pass's histograms by
+// every CTA (the same decision everywhere); digits 2-4 are counted per slice and the cluster's
+// histograms are summed through distributed shared memory. The compaction counts each slice's
+// keys > T and == T, takes the exclusive prefix over the lower ranks, and writes the slice's
+// indices from there: indices stay increasing and the kept ties are the lowest-indexed ones.
+__global__ void __cluster_dims__(kSelCluster, 1, 1) __launch_bounds__(kSelThreads)
+    select_topk_kernel(const SelectParams p) {
+  __shared__ int s_hist[256];      // this slice's histogram (read by the whole cluster)
+  __shared__ int s_hsum[256];      // the cluster's
   __shared__ int s_warp[33];
+  __shared__ int s_cnt[2];         // this slice's keys > T and == T (read by the whole cluster)
+  __shared__ int s_base[3];        // out position, ties before this slice, cluster total out
   __shared__ uint32_t s_prefix;
   __shared__ int s_need;
-  const int g = blockIdx.x, b = blockIdx.y;
+  uint32_t crank;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(crank));
+  const int rank = static_cast<int>(crank);
+  const int g = blockIdx.x / kSelCluster, b = blockIdx.y;
   const int tid = threadIdx.x;
   const int hi = sel_candidates(p, b);
   const long long bg = static_cast<long long>(b) * p.Hkv + g;
@@ -232,7 +262,8 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const SelectPa
   const uint4* keys4 = reinterpret_cast<const uint4*>(keys);
   int* out = p.sel + bg * p.n_sel;
   const int k = p.n_sel < hi ? p.n_sel : hi;   // fewer candidates than n_sel: keep them all
-  const int n4 = (hi + 3) >> 2;
+  const int per = (((hi + kSelCluster - 1) / kSelCluster) + 3) & ~3;   // slice length, 16-byte rows
+  const int lo = min(hi, rank * per), hi_c = min(hi, lo + per);
 
   // radix select: T = the k-th largest key; need = how many keys equal to T are kept
   uint32_t prefix = 0, mask = 0;
@@ -243,7 +274,7 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const SelectPa
       const int nch = (hi + kSelChunk - 1) / kSelChunk;
       const uint4* h4 = reinterpret_cast<const uint4*>(p.hist + bg * p.n_chunks * 256);
       const int lane = tid & 31, warp = tid >> 5;
-      if (tid < 256) s_hist[tid] = 0;
+      if (tid < 256) s_hsum[tid] = 0;
       int acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll 4
       for (int c = warp; c < nch; c += kSelThreads / 32) {
@@ -258,9 +289,9 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const SelectPa
       __syncthreads();
 #pragma unroll
       for (int e = 0; e < 8; ++e)
-        if (acc[e]) atomicAdd(&s_hist[8 * lane + e], acc[e]);
+        if (acc[e]) atomicAdd(&s_hsum[8 * lane + e], acc[e]);
       __syncthreads();
-      if (tid < 32) select_pick_bin(s_hist, 24, prefix, need, &s_prefix, &s_need);
+      if (tid < 32) select_pick_bin(s_hsum, 24, prefix, need, &s_prefix, &s_need);
       __syncthreads();
       prefix = s_prefix;
       need = s_need;
@@ -269,12 +300,12 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const SelectPa
     for (int shift = 16; shift >= 0; shift -= 8) {
       if (tid < 256) s_hist[tid] = 0;
       __syncthreads();
-      for (int i4 = tid; i4 < n4; i4 += kSelUnroll * kSelThreads) {
+      for (int i4 = (lo >> 2) + tid; i4 < (hi_c + 3) >> 2; i4 += kSelUnroll * kSelThreads) {
         uint4 v[kSelUnroll];
 #pragma unroll
         for (int r = 0; r < kSelUnroll; ++r) {
           const int j = i4 + r * kSelThreads;
-          v[r] = j < n4 ? keys4[j] : make_uint4(0u, 0u, 0u, 0u);
+          v[r] = j < (hi_c + 3) >> 2 ? keys4[j] : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
         for (int r = 0; r < kSelUnroll; ++r) {
@@ -282,39 +313,92 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const SelectPa
           const uint32_t u[4] = {v[r].x, v[r].y, v[r].z, v[r].w};
 #pragma unroll
           for (int e = 0; e < 4; ++e)
-            if (i0 + e < hi && (u[e] & mask) == prefix) atomicAdd(&s_hist[(u[e] >> shift) & 0xFFu], 1);
+            if (i0 + e < hi_c && (u[e] & mask) == prefix) atomicAdd(&s_hist[(u[e] >> shift) & 0xFFu], 1);
         }
       }
       __syncthreads();
-      if (tid < 32) select_pick_bin(s_hist, shift, prefix, need, &s_prefix, &s_need);
+      cluster_sync_all();   // every slice's histogram is complete and visible
+      if (tid < 256) {
+        int sum = 0;
+        for (int r = 0; r < kSelCluster; ++r) sum += ld_cluster_s32(cluster_map(smem_u32(&s_hist[tid]), r));
+        s_hsum[tid] = sum;
+      }
+      __syncthreads();
+      if (tid < 32) select_pick_bin(s_hsum, shift, prefix, need, &s_prefix, &s_need);
       __syncthreads();
       prefix = s_prefix;
       need = s_need;
       mask |= 0xFFu << shift;
+      cluster_sync_all();   // no CTA clears its histogram while another still reads it
     }
   }
   const bool take_all = k >= hi;
-  // ordered compaction, 16 consecutive candidates per thread: one block scan per step of the
-  // packed counts (keys == T in the high half, keys > T in the low half; each <= 16384)
-  int out_base = 0, tie_base = 0;
-  for (int base = 0; base < hi; base += kSelBlockKeys) {
-    const int i0 = base + kSelPerThread * tid;
-    uint4 v[kSelPerThread / 4];
-#pragma unroll
-    for (int r = 0; r < kSelPerThread / 4; ++r)
-      v[r] = i0 + 4 * r < hi ? keys4[(i0 >> 2) + r] : make_uint4(0u, 0u, 0u, 0u);
-    uint32_t gt = 0, eq = 0;   // bit e: candidate i0 + e
+  // per-slice counts of the keys kept outright (> T) and of the ties (== T)
+  auto classify = [&](int i0, const uint4 (&v)[kSelPerThread / 4], uint32_t& gt, uint32_t& eq) {
+    gt = 0;
+    eq = 0;
 #pragma unroll
     for (int r = 0; r < kSelPerThread / 4; ++r) {
       const uint32_t u[4] = {v[r].x, v[r].y, v[r].z, v[r].w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int idx = i0 + 4 * r + e;
-        const bool valid = idx < hi;
+        const bool valid = idx < hi_c;
         if (valid && (take_all || u[e] > prefix)) gt |= 1u << (4 * r + e);
         if (valid && !take_all && u[e] == prefix) eq |= 1u << (4 * r + e);
       }
     }
+  };
+  {
+    int ngt = 0, neq = 0;
+    for (int base = lo; base < hi_c; base += kSelBlockKeys) {
+      const int i0 = base + kSelPerThread * tid;
+      uint4 v[kSelPerThread / 4];
+#pragma unroll
+      for (int r = 0; r < kSelPerThread / 4; ++r)
+        v[r] = i0 + 4 * r < hi_c ? keys4[(i0 >> 2) + r] : make_uint4(0u, 0u, 0u, 0u);
+      uint32_t gt, eq;
+      classify(i0, v, gt, eq);
+      ngt += __popc(gt);
+      neq += __popc(eq);
+    }
+    int tg, te;   // two scans: a slice may hold more keys than a 16-bit field
+    block_exclusive_scan(ngt, tg, s_warp);
+    block_exclusive_scan(neq, te, s_warp);
+    if (tid == 0) {
+      s_cnt[0] = tg;
+      s_cnt[1] = te;
+    }
+  }
+  cluster_sync_all();       // every slice's counts are visible
+  if (tid == 0) {
+    int gt_before = 0, eq_before = 0, gt_all = 0, eq_all = 0;
+    for (int r = 0; r < kSelCluster; ++r) {
+      const int cg = ld_cluster_s32(cluster_map(smem_u32(&s_cnt[0]), r));
+      const int ce = ld_cluster_s32(cluster_map(smem_u32(&s_cnt[1]), r));
+      if (r < rank) {
+        gt_before += cg;
+        eq_before += ce;
+      }
+      gt_all += cg;
+      eq_all += ce;
+    }
+    s_base[0] = gt_before + (eq_before < need ? eq_before : need);
+    s_base[1] = eq_before;
+    s_base[2] = gt_all + (take_all ? 0 : (eq_all < need ? eq_all : need));
+  }
+  cluster_sync_all();       // the counts are read: a CTA may now finish and exit
+  // ordered compaction of the slice, 16 consecutive candidates per thread: one block scan per
+  // step of the packed counts (keys == T in the high half, keys > T in the low half)
+  int out_base = s_base[0], tie_base = s_base[1];
+  for (int base = lo; base < hi_c; base += kSelBlockKeys) {
+    const int i0 = base + kSelPerThread * tid;
+    uint4 v[kSelPerThread / 4];
+#pragma unroll
+    for (int r = 0; r < kSelPerThread / 4; ++r)
+      v[r] = i0 + 4 * r < hi_c ? keys4[(i0 >> 2) + r] : make_uint4(0u, 0u, 0u, 0u);
+    uint32_t gt, eq;
+    classify(i0, v, gt, eq);
     const int ngt = __popc(gt), neq = __popc(eq);
     int total;
     const int excl = block_exclusive_scan((neq << 16) | ngt, total, s_warp);
@@ -338,7 +422,8 @@ __global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const SelectPa
     out_base += (total & 0xFFFF) + (eq_total < rem ? eq_total : rem);
     tie_base += eq_total;
   }
-  for (int j = out_base + tid; j < p.n_sel; j += kSelThreads) out[j] = -1;   // too few candidates
+  if (rank == 0)
+    for (int j = s_base[2] + tid; j < p.n_sel; j += kSelThreads) out[j] = -1;   // too few candidates
 }
 
 }  // namespace mimo
