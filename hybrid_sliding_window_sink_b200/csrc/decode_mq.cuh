@@ -57,8 +57,14 @@ __device__ __forceinline__ int mq_range(const DecodeMqParams& p, int b, int& klo
   return L;
 }
 
-template <int G>
-__global__ void __launch_bounds__(kDecThreads, 2) decode_mq_kernel(const DecodeMqParams p) {
+// NW warps (16 rows each; NW * 16 >= T * G) and subtiles of SUB keys (64, or 32 for the ring
+// layers, whose 131-key units fit in a few subtiles: 40 KB of shared memory then lets five
+// CTAs share an SM).
+template <int G, int NW, int SUB>
+__global__ void __launch_bounds__(NW * 32) decode_mq_kernel(const DecodeMqParams p) {
+  constexpr int kThreads = NW * 32;
+  constexpr int kStageBytes = SUB * (kKRow + kVRow);
+  static_assert(SUB == 32 || SUB == 64, "subtile size");
   static_assert(G >= 1 && G <= 16, "group size");
   pdl_wait();
   pdl_trigger();
@@ -86,12 +92,12 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_mq_kernel(const DecodeM
   auto slot_of = [&](int tok) -> int { return p.mode == kModeRing ? tok % p.cap : tok; };
 
   auto load_sub = [&](int st, int stage) {
-    const uint32_t sK = s_base + stage * kDecStageBytes;
-    const uint32_t sV = sK + kDecSub * kKRow;
-    const int base = st * kDecSub;
+    const uint32_t sK = s_base + stage * kStageBytes;
+    const uint32_t sV = sK + SUB * kKRow;
+    const int base = st * SUB;
 #pragma unroll
-    for (int i = 0; i < (kDecSub * 24) / kDecThreads; ++i) {
-      const int idx = tid + i * kDecThreads;
+    for (int i = 0; i < (SUB * 24) / kThreads; ++i) {
+      const int idx = tid + i * kThreads;
       const int row = idx / 24, u = idx - row * 24;
       const int key = base + row;
       const bool ok = key < n_here;
@@ -100,8 +106,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_mq_kernel(const DecodeM
                  ok ? 16u : 0u);
     }
 #pragma unroll
-    for (int i = 0; i < (kDecSub * 16) / kDecThreads; ++i) {
-      const int idx = tid + i * kDecThreads;
+    for (int i = 0; i < (SUB * 16) / kThreads; ++i) {
+      const int idx = tid + i * kThreads;
       const int row = idx >> 4, u = idx & 15;
       const int key = base + row;
       const bool ok = key < n_here;
@@ -111,7 +117,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_mq_kernel(const DecodeM
     }
   };
 
-  const int nsub = (n_here + kDecSub - 1) / kDecSub;
+  const int nsub = (n_here + SUB - 1) / SUB;
   if (nsub > 0) load_sub(0, 0);
   cp_async_commit();
   if (nsub > 1) load_sub(1, 1);
@@ -155,15 +161,15 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_mq_kernel(const DecodeM
   for (int st = 0; st < nsub; ++st) {
     cp_async_wait<1>();
     __syncthreads();
-    const uint32_t sK = s_base + (st & 1) * kDecStageBytes;
-    const uint32_t sV = sK + kDecSub * kKRow;
+    const uint32_t sK = s_base + (st & 1) * kStageBytes;
+    const uint32_t sV = sK + SUB * kKRow;
     if (active) {
       // S = Q K^T over the 64 keys of the subtile (eight n-tiles of 8 keys)
-      float sacc[8][4];
+      float sacc[SUB / 8][4];
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+      for (int nt = 0; nt < SUB / 8; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
 #pragma unroll
-      for (int kg = 0; kg < 4; ++kg) {
+      for (int kg = 0; kg < SUB / 16; ++kg) {
         const int krow = kg * 16 + ((mi >> 1) << 3) + r8;
         const uint32_t rowaddr = sK + krow * kKRow;
 #pragma unroll
@@ -176,13 +182,13 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_mq_kernel(const DecodeM
         }
       }
       // mask by each row's key interval, online softmax (log2 domain)
-      const int tokbase = tok0 + st * kDecSub + tq * 2;
+      const int tokbase = tok0 + st * SUB + tq * 2;
       float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
+      for (int nt = 0; nt < SUB / 8; ++nt) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int key = st * kDecSub + nt * 8 + tq * 2 + (e & 1);
+          const int key = st * SUB + nt * 8 + tq * 2 + (e & 1);
           const int tok = tokbase + nt * 8 + (e & 1);
           const bool in = key < n_here && (e < 2 ? (tok >= lo0 && tok <= hi0) : (tok >= lo1 && tok <= hi1));
           sacc[nt][e] = in ? sacc[nt][e] * p.scale_log2 : -INFINITY;
@@ -199,9 +205,9 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_mq_kernel(const DecodeM
       const float ref1 = mn1 == -INFINITY ? 0.f : mn1;
       const float al0 = ex2(m0 - ref0), al1 = ex2(m1 - ref1);
       float s0 = 0.f, s1 = 0.f;
-      uint32_t pa[4][4];
+      uint32_t pa[SUB / 16][4];
 #pragma unroll
-      for (int kg = 0; kg < 4; ++kg) {
+      for (int kg = 0; kg < SUB / 16; ++kg) {
         float pv[2][4];
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
@@ -228,7 +234,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_mq_kernel(const DecodeM
       }
       // O += P V, 16 keys per k-step
 #pragma unroll
-      for (int kg = 0; kg < 4; ++kg) {
+      for (int kg = 0; kg < SUB / 16; ++kg) {
         const int vrow = kg * 16 + ((mi & 1) << 3) + r8;
         const uint32_t rowaddr = sV + vrow * kVRow;
 #pragma unroll

@@ -642,18 +642,20 @@ mimo_status launch_decode_mq_tma_g(const mimo::DecodeMqParams& prm, cudaStream_t
   return MIMO_OK;
 }
 
-template <int G>
-mimo_status launch_decode_mq_g(const mimo::DecodeMqParams& prm, cudaStream_t st) {
-  if (prm.mode == mimo::kModeLinear) return launch_decode_mq_tma_g<G>(prm, st);
-  auto kern = mimo::decode_mq_kernel<G>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, mimo::kDecSmemBytes) !=
-      cudaSuccess) {
+// Ring caches: decode_mq_kernel with 32-key subtiles (two stages: 40 KB of shared memory) and
+// as many warps as 16-row tiles of the T * G rows (2 for the MTP step's SWA layers, 4 above 32
+// rows), so the 131-slot units of a layer fit in one wave.
+template <int G, int NW>
+mimo_status launch_decode_mq_ring(const mimo::DecodeMqParams& prm, cudaStream_t st) {
+  constexpr int kSub = 32;
+  auto kern = mimo::decode_mq_kernel<G, NW, kSub>;
+  const int smem = 2 * kSub * (mimo::kKRow + mimo::kVRow);
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
     cudaGetLastError();
     return MIMO_ERR_CUDA;
   }
   dim3 grid(prm.nchunks, prm.Hkv, prm.B);
-  if (launch_pdl(kern, grid, mimo::kDecThreads, mimo::kDecSmemBytes, st, prm, false) != cudaSuccess)
-    return MIMO_ERR_CUDA;
+  if (launch_pdl(kern, grid, NW * 32, smem, st, prm, false) != cudaSuccess) return MIMO_ERR_CUDA;
   if (!prm.direct) {
     const long long rows = static_cast<long long>(prm.B) * prm.T * prm.Hq;
     if (rows > 0x7fffffffLL) return MIMO_ERR_UNSUPPORTED;
@@ -662,6 +664,13 @@ mimo_status launch_decode_mq_g(const mimo::DecodeMqParams& prm, cudaStream_t st)
       return MIMO_ERR_CUDA;
   }
   return MIMO_OK;
+}
+
+template <int G>
+mimo_status launch_decode_mq_g(const mimo::DecodeMqParams& prm, cudaStream_t st) {
+  if (prm.mode == mimo::kModeLinear) return launch_decode_mq_tma_g<G>(prm, st);
+  if (prm.T * G <= 32) return launch_decode_mq_ring<G, 2>(prm, st);
+  return launch_decode_mq_ring<G, 4>(prm, st);
 }
 
 }  // namespace
