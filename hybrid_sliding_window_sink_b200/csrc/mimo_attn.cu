@@ -590,9 +590,11 @@ DecodePlan plan_decode_mq(const mimo_shape* s, int mode, int cap, int T, int W, 
   if (total <= 256) {
     pl.chunk = static_cast<int>((total + 63) / 64 * 64);
   } else {
+    // linear caches: long chunks, since each CTA of the TMA kernel holds an SM and drains its
+    // pipeline at the end (8192-key chunks measured 2% faster than 4096, 2048 slower)
     const long long c = total * units / (16LL * sms);
     const int ch = pow2_floor(c);
-    pl.chunk = ch < 256 ? 256 : (ch > 4096 ? 4096 : ch);
+    pl.chunk = ch < 256 ? 256 : (ch > 8192 ? 8192 : ch);
   }
   pl.nchunks = static_cast<int>((total + pl.chunk - 1) / pl.chunk);
   pl.direct = pl.nchunks == 1;
@@ -875,7 +877,25 @@ mimo_status mimo_attn_select_tokens(const mimo_shape* s, const void* q, const vo
   }
   if (!launched) return MIMO_ERR_CUDA;
   if (cudaGetLastError() != cudaSuccess) return MIMO_ERR_CUDA;
-  mimo::select_topk_kernel<<<dim3(s->n_kv_heads * mimo::kSelCluster, s->batch), mimo::kSelThreads, 0, st>>>(prm);
+  // top-k: a cluster of kSelCluster CTAs per (b, g) for long caches (each slice then holds
+  // tens of thousands of keys), one CTA per (b, g) below that (small slices cost more in
+  // cluster barriers and loop overhead than they save)
+  if (cache_capacity >= mimo::kSelClusterMinCap) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(s->n_kv_heads * mimo::kSelCluster, s->batch);
+    cfg.blockDim = dim3(mimo::kSelThreads);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = mimo::kSelCluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, mimo::select_topk_kernel<mimo::kSelCluster>, prm) != cudaSuccess) return MIMO_ERR_CUDA;
+  } else {
+    mimo::select_topk_kernel<1><<<dim3(s->n_kv_heads, s->batch), mimo::kSelThreads, 0, st>>>(prm);
+  }
   return cudaGetLastError() == cudaSuccess ? MIMO_OK : MIMO_ERR_CUDA;
 }
 

@@ -27,7 +27,8 @@ constexpr int kSelThreads = 1024;
 constexpr int kSelPerThread = 16;                 // candidates per thread per compaction step
 constexpr int kSelBlockKeys = kSelPerThread * kSelThreads;
 constexpr int kSelUnroll = 8;                     // 16-byte key loads in flight per thread
-constexpr int kSelCluster = 8;                    // CTAs per (b, g) in the top-k
+constexpr int kSelCluster = 8;                    // CTAs per (b, g) in the top-k of long caches
+constexpr int kSelClusterMinCap = 131072;         // capacity from which the top-k uses clusters
 
 struct SelectParams {
   const __nv_bfloat16* q;     // [B, Hq, 192]
@@ -236,14 +237,15 @@ __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
 }
 
-// Top-k per (b, g) on a cluster of kSelCluster CTAs: CTA `rank` owns the contiguous candidate
+// Top-k per (b, g) on a cluster of CS CTAs (launched with that cluster size; CS = 1 is one CTA
+// per (b, g)): CTA `rank` owns the contiguous candidate
 // slice [lo, hi_c). Digit 1 of the radix select is summed from the score pass's histograms by
 // every CTA (the same decision everywhere); digits 2-4 are counted per slice and the cluster's
 // histograms are summed through distributed shared memory. The compaction counts each slice's
 // keys > T and == T, takes the exclusive prefix over the lower ranks, and writes the slice's
 // indices from there: indices stay increasing and the kept ties are the lowest-indexed ones.
-__global__ void __cluster_dims__(kSelCluster, 1, 1) __launch_bounds__(kSelThreads)
-    select_topk_kernel(const SelectParams p) {
+template <int CS>
+__global__ void __launch_bounds__(kSelThreads) select_topk_kernel(const SelectParams p) {
   __shared__ int s_hist[256];      // this slice's histogram (read by the whole cluster)
   __shared__ int s_hsum[256];      // the cluster's
   __shared__ int s_warp[33];
@@ -254,7 +256,7 @@ __global__ void __cluster_dims__(kSelCluster, 1, 1) __launch_bounds__(kSelThread
   uint32_t crank;
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(crank));
   const int rank = static_cast<int>(crank);
-  const int g = blockIdx.x / kSelCluster, b = blockIdx.y;
+  const int g = blockIdx.x / CS, b = blockIdx.y;
   const int tid = threadIdx.x;
   const int hi = sel_candidates(p, b);
   const long long bg = static_cast<long long>(b) * p.Hkv + g;
@@ -262,7 +264,7 @@ __global__ void __cluster_dims__(kSelCluster, 1, 1) __launch_bounds__(kSelThread
   const uint4* keys4 = reinterpret_cast<const uint4*>(keys);
   int* out = p.sel + bg * p.n_sel;
   const int k = p.n_sel < hi ? p.n_sel : hi;   // fewer candidates than n_sel: keep them all
-  const int per = (((hi + kSelCluster - 1) / kSelCluster) + 3) & ~3;   // slice length, 16-byte rows
+  const int per = (((hi + CS - 1) / CS) + 3) & ~3;   // slice length, 16-byte rows
   const int lo = min(hi, rank * per), hi_c = min(hi, lo + per);
 
   // radix select: T = the k-th largest key; need = how many keys equal to T are kept
@@ -320,7 +322,7 @@ __global__ void __cluster_dims__(kSelCluster, 1, 1) __launch_bounds__(kSelThread
       cluster_sync_all();   // every slice's histogram is complete and visible
       if (tid < 256) {
         int sum = 0;
-        for (int r = 0; r < kSelCluster; ++r) sum += ld_cluster_s32(cluster_map(smem_u32(&s_hist[tid]), r));
+        for (int r = 0; r < CS; ++r) sum += ld_cluster_s32(cluster_map(smem_u32(&s_hist[tid]), r));
         s_hsum[tid] = sum;
       }
       __syncthreads();
@@ -373,7 +375,7 @@ __global__ void __cluster_dims__(kSelCluster, 1, 1) __launch_bounds__(kSelThread
   cluster_sync_all();       // every slice's counts are visible
   if (tid == 0) {
     int gt_before = 0, eq_before = 0, gt_all = 0, eq_all = 0;
-    for (int r = 0; r < kSelCluster; ++r) {
+    for (int r = 0; r < CS; ++r) {
       const int cg = ld_cluster_s32(cluster_map(smem_u32(&s_cnt[0]), r));
       const int ce = ld_cluster_s32(cluster_map(smem_u32(&s_cnt[1]), r));
       if (r < rank) {

@@ -63,8 +63,8 @@ def test_wait_on_a_barrier_nothing_arrives_on(cuda_device):
 
 def test_kernels_give_up_and_the_context_stays_usable(cuda_device):
     """Under the 1 ns wait limit the persistent SWA-ring and GA-pair prefill kernels give up
-    (wait-timeout bit) and the generic prefill and decode kernels may (their waits are short);
-    no exit-path wait ever gives up. Afterwards the product build, on the same context,
+    (wait-timeout bit) and the generic prefill, decode and multi-query decode kernels may (their
+    waits are short); no exit-path wait ever gives up. Afterwards the product build, on the same context,
     matches the oracle and leaves the word clear."""
     dev = cuda_device
     cases = [(wl.prefill_inputs(1, 640, 64, 8, seed=61), 128, 1e4),             # SWA ring kernel
@@ -73,6 +73,9 @@ def test_kernels_give_up_and_the_context_stays_usable(cuda_device):
     lengths = [4096, 100, 3000, 1, 4096, 2048, 7, 999]
     d = wl.decode_inputs(len(lengths), 64, 4, 4096, lengths, seed=64)
     dd = {k: v.to(dev) for k, v in d.items()}
+    mq_lengths = [3000, 4, 1500]    # multi-query decode over a linear cache: the TMA / tcgen05 kernel
+    mq = wl.decode_mq_inputs(len(mq_lengths), 4, 64, 4, 3000, mq_lengths, seed=66)
+    mqd = {k: v.to(dev) for k, v in mq.items()}
     with _library("shortwait") as lib:
         for i, (x, window, theta) in enumerate(cases):
             _lib.prefill(x["q"].to(dev), x["k"].to(dev), x["v"].to(dev), x["sink"].to(dev),
@@ -82,6 +85,10 @@ def test_kernels_give_up_and_the_context_stays_usable(cuda_device):
             if i < 2:   # persistent kernels: every CTA waits on work in progress many times
                 assert word == WAIT_TIMEOUT, (window, word)
         _lib.decode(dd["q"], dd["k_cache"], dd["v_cache"], dd["lengths"], dd["sink"], kind="linear")
+        st, word = _status(lib)
+        assert not word & DRAIN_TIMEOUT, word
+        _lib.decode_mq(mqd["q_mq"], mqd["k_cache"], mqd["v_cache"], mqd["lengths"], mqd["sink"], kind="linear",
+                       window=0)
         st, word = _status(lib)
         assert not word & DRAIN_TIMEOUT, word
     for x, window, theta in cases:
@@ -96,6 +103,12 @@ def test_kernels_give_up_and_the_context_stays_usable(cuda_device):
     o_ref, l_ref = ref.decode(wl.to_f64(d["q"]), wl.to_f64(d["k_cache"]), wl.to_f64(d["v_cache"]), "linear",
                               lengths, wl.to_f64(d["sink"]))
     compare(wl.to_f64(out), o_ref, wl.to_f64(lse), l_ref, "after abort: decode")
+    out, lse = _lib.decode_mq(mqd["q_mq"], mqd["k_cache"], mqd["v_cache"], mqd["lengths"], mqd["sink"],
+                              kind="linear", window=0)
+    torch.cuda.synchronize()
+    o_ref, l_ref = ref.decode_multi(wl.to_f64(mq["q_mq"]), wl.to_f64(mq["k_cache"]), wl.to_f64(mq["v_cache"]),
+                                    "linear", mq_lengths, 0, wl.to_f64(mq["sink"]))
+    compare(wl.to_f64(out), o_ref, wl.to_f64(lse), l_ref, "after abort: multi-query decode")
     assert _status(_lib.lib()) == (MIMO_OK, 0)
 
 
