@@ -322,32 +322,58 @@ def bench_chunk_prefill(steps, warmup, peaks, tag, dev, stream, chunk=16384, pre
 
 
 def e2e_prefill(case, steps, dev, stream):
-    """Same metric through the public call with host buffers: pinned H2D of the step's
-    inputs, the kernel, D2H of the outputs, all inside the timed region."""
+    """Same metric through the public call with host buffers: every step copies its inputs from
+    pinned host memory to the device, runs the call and copies out and lse back, all inside the
+    timed region. Steps are pipelined the way a serving loop would run them: the host-to-device
+    copies of step i + 1 and the device-to-host copies of step i - 1 overlap the call of step i
+    (three streams, two device buffer sets; PCIe carries both directions at once)."""
     from hybrid_sliding_window_sink_b200 import _lib
     host = wl.case_prefill_inputs(case, device="cpu")
     host = {k: v.pin_memory() for k, v in host.items()}
-    dq = torch.empty_like(host["q"], device=dev)
-    dk = torch.empty_like(host["k"], device=dev)
-    dv = torch.empty_like(host["v"], device=dev)
-    ds = torch.empty_like(host["sink"], device=dev)
-    out = torch.empty(case.batch, case.seqlen, case.hq, wl.DV, dtype=torch.bfloat16, device=dev)
-    lse = torch.empty(case.batch, case.hq, case.seqlen, dtype=torch.float32, device=dev)
-    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    h_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    sets = []
+    for _ in range(2):
+        sets.append({
+            "q": torch.empty_like(host["q"], device=dev), "k": torch.empty_like(host["k"], device=dev),
+            "v": torch.empty_like(host["v"], device=dev), "sink": torch.empty_like(host["sink"], device=dev),
+            "out": torch.empty(case.batch, case.seqlen, case.hq, wl.DV, dtype=torch.bfloat16, device=dev),
+            "lse": torch.empty(case.batch, case.hq, case.seqlen, dtype=torch.float32, device=dev)})
+    h_out = torch.empty(sets[0]["out"].shape, dtype=torch.bfloat16).pin_memory()
+    h_lse = torch.empty(sets[0]["lse"].shape, dtype=torch.float32).pin_memory()
+    s_in, s_cmp, s_out = torch.cuda.Stream(device=dev), stream, torch.cuda.Stream(device=dev)
+    ev = {name: [torch.cuda.Event() for _ in range(2)] for name in ("in", "cmp", "out")}
+    started = [False, False]
 
-    def step():
-        with torch.cuda.stream(stream):
-            dq.copy_(host["q"], non_blocking=True)
-            dk.copy_(host["k"], non_blocking=True)
-            dv.copy_(host["v"], non_blocking=True)
-            ds.copy_(host["sink"], non_blocking=True)
-            _lib.prefill(dq, dk, dv, ds, window=case.window, rope_theta=case.theta,
-                         rot_dims=wl.ROT_DIMS, out=out, lse=lse, stream=stream)
-            h_out.copy_(out, non_blocking=True)
-            h_lse.copy_(lse, non_blocking=True)
+    def step(i):
+        b, d = i % 2, sets[i % 2]
+        with torch.cuda.stream(s_in):
+            if started[b]:
+                s_in.wait_event(ev["cmp"][b])          # step i - 2 has read this input set
+            for name in ("q", "k", "v", "sink"):
+                d[name].copy_(host[name], non_blocking=True)
+            ev["in"][b].record(s_in)
+        s_cmp.wait_event(ev["in"][b])
+        if started[b]:
+            s_cmp.wait_event(ev["out"][b])             # step i - 2's outputs have left this set
+        _lib.prefill(d["q"], d["k"], d["v"], d["sink"], window=case.window, rope_theta=case.theta,
+                     rot_dims=wl.ROT_DIMS, out=d["out"], lse=d["lse"], stream=s_cmp)
+        ev["cmp"][b].record(s_cmp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev["cmp"][b])
+            h_out.copy_(d["out"], non_blocking=True)
+            h_lse.copy_(d["lse"], non_blocking=True)
+            ev["out"][b].record(s_out)
+        started[b] = True
 
-    ms = timed(step, steps, 1, stream)
+    for i in range(3):                                 # warm-up: both buffer sets, then one more
+        step(i)
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(s_in)
+    for i in range(steps):
+        step(i)
+    t1.record(s_out)                                   # after the last step's copies out
+    torch.cuda.synchronize(dev)
+    ms = t0.elapsed_time(t1)
     h2d = sum(t.numel() * t.element_size() for t in host.values())
     d2h = h_out.numel() * h_out.element_size() + h_lse.numel() * h_lse.element_size()
     return ms / steps, h2d, d2h
@@ -763,7 +789,7 @@ def main():
     ap.add_argument("--impl", default="mimo", choices=["mimo", "reference"])
     ap.add_argument("--only-main", action="store_true", help="skip the extra workloads")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=8)
     ap.add_argument("--detail", default=None, help="also write the full per-workload records here")
     ap.add_argument("--decode-shard", action="store_true",
                     help="time only the 48-layer decode step, its 64 sequences partitioned across ranks")
