@@ -31,6 +31,21 @@
 
 namespace mimo {
 
+// Optional per-tile timestamps (debug builds with -DMIMO_TRACE; compiled out otherwise):
+// events 0/1 S issued (group A/B), 2/3 PV issued, 4/5 S seen by the softmax group, 6/7 P
+// written, 9 K tile rotated, 10/11 S issue started, 12/13 PV issue started.
+#ifdef MIMO_TRACE
+#define GA_TRACE(tile, ev)                                                             \
+  do {                                                                                 \
+    if (p.trace && blockIdx.x < 8 && (tile) < 256)                                     \
+      p.trace[(static_cast<size_t>(blockIdx.x) * 256 + (tile)) * 32 + (ev)] = clock64(); \
+  } while (0)
+#else
+#define GA_TRACE(tile, ev) \
+  do {                     \
+  } while (0)
+#endif
+
 // 32 consecutive TMEM columns of this warp's 32 lanes.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   tmem_ld16(taddr, *reinterpret_cast<uint32_t(*)[16]>(r));
@@ -225,6 +240,7 @@ __global__ void __launch_bounds__(kGaThreads, 1)
           if (ready && s_gt >= 1) ready = mbar_test(bar(kGaPVDone + s_grp), (s_gt - 1) & 1);
           if (ready) {
             tc_fence_after();
+            GA_TRACE(s_gt, 10 + s_grp);
             const uint32_t d = tmem + s_grp * 256;
             const uint32_t kb = sK + (s_gt & 1) * L::K_TILE;
 #pragma unroll
@@ -234,6 +250,7 @@ __global__ void __launch_bounds__(kGaThreads, 1)
               umma_ss(d, a, bd, kk * 16 < p.rot_dims ? L::IDESC_S_F16 : L::IDESC_S, kk > 0 ? 1u : 0u);
             }
             umma_commit(bar(kGaSFull + s_grp));
+            GA_TRACE(s_gt, s_grp);
             if (s_grp == 1) {
               umma_commit(bar(kGaKEmpty + (s_gt & 1)));
               if (s_j == s_T - 1) umma_commit(bar(kGaQEmpty));
@@ -257,6 +274,7 @@ __global__ void __launch_bounds__(kGaThreads, 1)
           if (ready && v_grp == 0) ready = mbar_test(bar(kGaVFull), v_gt & 1);
           if (ready) {
             tc_fence_after();
+            GA_TRACE(v_gt, 12 + v_grp);
             const uint32_t base = tmem + v_grp * 256;
 #pragma unroll
             for (int s2 = 0; s2 < kGaBN / 16; ++s2) {
@@ -264,6 +282,7 @@ __global__ void __launch_bounds__(kGaThreads, 1)
               umma_ts(base + 128, base + 8 * s2, bd, L::IDESC_PV, (v_j > 0 || s2 > 0) ? 1u : 0u);
             }
             umma_commit(bar(kGaPVDone + v_grp));
+            GA_TRACE(v_gt, 2 + v_grp);
             if (v_grp == 1) {
               umma_commit(bar(kGaVEmpty));
               v_grp = 0;
@@ -400,6 +419,7 @@ __global__ void __launch_bounds__(kGaThreads, 1)
           if (!wait_all(bar(kGaKFull + ks), (gt >> 1) & 1)) { ok = false; break; }
         }
         mbar_arrive(bar(kGaKReady + ks));
+        if (ctid == 0) GA_TRACE(gt, 9);
       }
     }
   } else {
@@ -428,6 +448,7 @@ __global__ void __launch_bounds__(kGaThreads, 1)
       for (int j = 0; j < T; ++j, ++gt) {
         if (!wait_all(bar(kGaSFull + grp), gt & 1)) { ok = false; break; }
         tc_fence_after();
+        if (q4 == 0 && lane == 0) GA_TRACE(gt, 4 + grp);
         const int kt0 = j * kGaBN;
         const bool full = kt0 + kGaBN - 1 <= pmin;   // every key of the tile is <= every row's pos
         // pass 1: tile max of the valid keys, 64 columns per TMEM round trip
@@ -520,6 +541,7 @@ __global__ void __launch_bounds__(kGaThreads, 1)
           pass2(std::true_type{});
         tmem_wait_st();
         tc_fence_before();
+        if (q4 == 0 && lane == 0) GA_TRACE(gt, 6 + grp);
         mbar_arrive(bar(kGaPReady + grp));
         const float2 s2 = f2_unpack(sab);
         l += s2.x + s2.y;
