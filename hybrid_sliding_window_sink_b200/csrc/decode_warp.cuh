@@ -32,27 +32,30 @@ constexpr int kDwMaxStages = 3;
 __host__ __device__ constexpr int dw_smem_bytes(int stages) { return stages * (kDwStageBytes + kDwKeys * 4); }
 
 // The warp copies 32 K and V rows (tokens tk[0..31] of one sequence and KV head; a negative
-// token is zero-filled) into a stage by 16-byte cp.async: 24 + 16 chunks per lane, K rows
-// XOR-swizzled for ldmatrix. The caller commits the group.
+// token is zero-filled) into a stage by 16-byte cp.async, K rows XOR-swizzled for ldmatrix.
+// Lane l serves rows 4 i + l / 8 (i = 0..7) and, in each, the 16-byte units 8 p + l % 8: every
+// warp instruction reads 128 contiguous bytes from each of 4 rows, and a lane resolves each of
+// its rows (token, global and shared addresses) once for all of that row's units. The caller
+// commits the group.
 __device__ __forceinline__ void dw_gather(uint32_t sK, uint32_t sV, const int* tk, const __nv_bfloat16* kbase,
                                           const __nv_bfloat16* vbase, long long seq0, long long krow_stride,
                                           long long vrow_stride) {
-  const int lane = threadIdx.x & 31;
-#pragma unroll 8
-  for (int i = 0; i < 24; ++i) {                   // 32 rows x 24 chunks of K
-    const int idx = lane + 32 * i;
-    const int row = idx / 24, u = idx - row * 24;
+  const int lane = threadIdx.x & 31, lr = lane >> 3, lu = lane & 7;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int row = 4 * i + lr;
     const int t = tk[row];
-    cp_async16(sK + row * kKRow + ((u ^ (row & 7)) << 4),
-               kbase + (seq0 + (t < 0 ? 0 : t)) * krow_stride + u * 8, t < 0 ? 0u : 16u);
-  }
-#pragma unroll 8
-  for (int i = 0; i < 16; ++i) {                   // 32 rows x 16 chunks of V
-    const int idx = lane + 32 * i;
-    const int row = idx >> 4, u = idx & 15;
-    const int t = tk[row];
-    cp_async16(sV + row * kVRow + ((u ^ (row & 7)) << 4),
-               vbase + (seq0 + (t < 0 ? 0 : t)) * vrow_stride + u * 8, t < 0 ? 0u : 16u);
+    const uint32_t sz = t < 0 ? 0u : 16u;
+    const long long tok = seq0 + (t < 0 ? 0 : t);
+    const __nv_bfloat16* kg = kbase + tok * krow_stride + lu * 8;
+    const __nv_bfloat16* vg = vbase + tok * vrow_stride + lu * 8;
+    // unit 8 p + lu lands at unit 8 p + (lu ^ (row & 7)) of the row (the XOR keeps the low 3 bits)
+    const uint32_t sw = static_cast<uint32_t>((lu ^ (row & 7)) << 4);
+    const uint32_t sk = sK + row * kKRow + sw, sv = sV + row * kVRow + sw;
+#pragma unroll
+    for (int pp = 0; pp < kKRow / 128; ++pp) cp_async16(sk + pp * 128, kg + pp * 64, sz);
+#pragma unroll
+    for (int pp = 0; pp < kVRow / 128; ++pp) cp_async16(sv + pp * 128, vg + pp * 64, sz);
   }
 }
 
