@@ -157,31 +157,30 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_split_kernel(const Deco
     return p.mode == kModeSparse ? s_tok[key] : k_begin + key;
   };
 
+  // Thread t serves rows 16 i + t / 8 of the subtile and, in each, the 16-byte units 8 p + t % 8:
+  // every warp instruction reads 128 contiguous bytes from each of 4 rows, and a row (token,
+  // global and shared addresses) is resolved once for all of its units.
   auto load_sub = [&](int st, int stage) {
     const uint32_t sK = s_base + stage * kDecStageBytes;
     const uint32_t sV = sK + kDecSub * kKRow;
     const int base = st * kDecSub;
+    const int lr = tid >> 3, lu = tid & 7;
 #pragma unroll
-    for (int i = 0; i < (kDecSub * 24) / kDecThreads; ++i) {     // 12 x 16 B of K per thread
-      const int idx = tid + i * kDecThreads;
-      const int row = idx / 24, u = idx - row * 24;
+    for (int i = 0; i < kDecSub / (kDecThreads / 8); ++i) {
+      const int row = (kDecThreads / 8) * i + lr;
       const int key = base + row;
       int tok = key < n_here ? token_of(key) : -1;
-      const bool ok = tok >= 0;
-      tok = ok ? tok : 0;
-      const __nv_bfloat16* src = kbase + (seq0 + tok) * krow_stride + u * 8;
-      cp_async16(sK + row * kKRow + ((u ^ (row & 7)) << 4), src, ok ? 16u : 0u);
-    }
+      const uint32_t sz = tok >= 0 ? 16u : 0u;
+      tok = tok >= 0 ? tok : 0;
+      const __nv_bfloat16* kg = kbase + (seq0 + tok) * krow_stride + lu * 8;
+      const __nv_bfloat16* vg = vbase + (seq0 + tok) * vrow_stride + lu * 8;
+      // unit 8 p + lu lands at unit 8 p + (lu ^ (row & 7)) (the XOR keeps the low 3 bits)
+      const uint32_t sw = static_cast<uint32_t>((lu ^ (row & 7)) << 4);
+      const uint32_t sk = sK + row * kKRow + sw, sv = sV + row * kVRow + sw;
 #pragma unroll
-    for (int i = 0; i < (kDecSub * 16) / kDecThreads; ++i) {     // 8 x 16 B of V per thread
-      const int idx = tid + i * kDecThreads;
-      const int row = idx >> 4, u = idx & 15;
-      const int key = base + row;
-      int tok = key < n_here ? token_of(key) : -1;
-      const bool ok = tok >= 0;
-      tok = ok ? tok : 0;
-      const __nv_bfloat16* src = vbase + (seq0 + tok) * vrow_stride + u * 8;
-      cp_async16(sV + row * kVRow + ((u ^ (row & 7)) << 4), src, ok ? 16u : 0u);
+      for (int pp = 0; pp < kKRow / 128; ++pp) cp_async16(sk + pp * 128, kg + pp * 64, sz);
+#pragma unroll
+      for (int pp = 0; pp < kVRow / 128; ++pp) cp_async16(sv + pp * 128, vg + pp * 64, sz);
     }
   };
 

@@ -48,28 +48,29 @@ __host__ __device__ constexpr int d8_smem_bytes(int stages) { return stages * (k
 
 // The warp copies the K and V bytes and the two scales of 32 keys (tokens tk[0..31] of one
 // sequence and KV head; a negative token is zero-filled) into a stage at sK: K rows as they
-// are, V rows XOR-swizzled in 16-byte units, then ks[32] and vs[32]. 22 cp.async per lane;
-// the caller commits the group.
+// are, V rows XOR-swizzled in 16-byte units, then ks[32] and vs[32]. Lane l serves rows
+// 8 i + l / 4 (i = 0..3) and, in each, the 16-byte units 4 j + l % 4: every warp instruction
+// reads 64 contiguous bytes from each of 8 rows, and a lane resolves each of its rows once.
+// 22 cp.async per lane; the caller commits the group.
 __device__ __forceinline__ void d8_gather(uint32_t sK, const int* tk, const uint8_t* kbase, const uint8_t* vbase,
                                           const float* ksbase, const float* vsbase, long long seq0,
                                           long long krow_stride, long long vrow_stride, int hkv) {
-  const int lane = threadIdx.x & 31;
+  const int lane = threadIdx.x & 31, lr = lane >> 2, lu = lane & 3;
   const uint32_t sV = sK + kD8KBytes, sS = sV + kD8VBytes;
 #pragma unroll
-  for (int i = 0; i < 12; ++i) {                   // 32 rows x 12 chunks of K
-    const int idx = lane + 32 * i;
-    const int row = idx / 12, u = idx - row * 12;
+  for (int i = 0; i < 4; ++i) {
+    const int row = 8 * i + lr;
     const int t = tk[row];
-    cp_async16(sK + row * kKRow8 + u * 16, kbase + (seq0 + (t < 0 ? 0 : t)) * krow_stride + u * 16,
-               t < 0 ? 0u : 16u);
-  }
+    const uint32_t sz = t < 0 ? 0u : 16u;
+    const long long tok = seq0 + (t < 0 ? 0 : t);
+    const uint8_t* kg = kbase + tok * krow_stride + lu * 16;
+    const uint8_t* vg = vbase + tok * vrow_stride + lu * 16;
+    const uint32_t sk = sK + row * kKRow8 + lu * 16;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {                    // 32 rows x 8 chunks of V
-    const int idx = lane + 32 * i;
-    const int row = idx >> 3, u = idx & 7;
-    const int t = tk[row];
-    cp_async16(sV + row * kVRow8 + ((u ^ (row & 7)) << 4), vbase + (seq0 + (t < 0 ? 0 : t)) * vrow_stride + u * 16,
-               t < 0 ? 0u : 16u);
+    for (int j = 0; j < kKRow8 / 64; ++j) cp_async16(sk + j * 64, kg + j * 64, sz);
+#pragma unroll
+    for (int j = 0; j < kVRow8 / 64; ++j)
+      cp_async16(sV + row * kVRow8 + (((4 * j + lu) ^ (row & 7)) << 4), vg + j * 64, sz);
   }
   const int t = tk[lane];                          // the two scales of key `lane`
   const long long srow = (seq0 + (t < 0 ? 0 : t)) * hkv;

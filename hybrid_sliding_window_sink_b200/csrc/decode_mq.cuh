@@ -91,29 +91,31 @@ __global__ void __launch_bounds__(NW * 32) decode_mq_kernel(const DecodeMqParams
   const long long vrow_stride = static_cast<long long>(p.Hkv) * kDV;
   auto slot_of = [&](int tok) -> int { return p.mode == kModeRing ? tok % p.cap : tok; };
 
+  // Thread t serves rows (kThreads / 8) i + t / 8 of the subtile and, in each, the 16-byte units
+  // 8 p + t % 8: every warp instruction reads 128 contiguous bytes from each of 4 rows, and a
+  // row (slot, global and shared addresses) is resolved once for all of its units.
+  static_assert(SUB % (kThreads / 8) == 0, "rows per pass");
   auto load_sub = [&](int st, int stage) {
     const uint32_t sK = s_base + stage * kStageBytes;
     const uint32_t sV = sK + SUB * kKRow;
     const int base = st * SUB;
+    const int lr = tid >> 3, lu = tid & 7;
 #pragma unroll
-    for (int i = 0; i < (SUB * 24) / kThreads; ++i) {
-      const int idx = tid + i * kThreads;
-      const int row = idx / 24, u = idx - row * 24;
+    for (int i = 0; i < SUB / (kThreads / 8); ++i) {
+      const int row = (kThreads / 8) * i + lr;
       const int key = base + row;
       const bool ok = key < n_here;
       const int slot = ok ? slot_of(tok0 + key) : 0;
-      cp_async16(sK + row * kKRow + ((u ^ (row & 7)) << 4), kbase + (seq0 + slot) * krow_stride + u * 8,
-                 ok ? 16u : 0u);
-    }
+      const uint32_t sz = ok ? 16u : 0u;
+      const __nv_bfloat16* kg = kbase + (seq0 + slot) * krow_stride + lu * 8;
+      const __nv_bfloat16* vg = vbase + (seq0 + slot) * vrow_stride + lu * 8;
+      // unit 8 p + lu lands at unit 8 p + (lu ^ (row & 7)) (the XOR keeps the low 3 bits)
+      const uint32_t sw = static_cast<uint32_t>((lu ^ (row & 7)) << 4);
+      const uint32_t sk = sK + row * kKRow + sw, sv = sV + row * kVRow + sw;
 #pragma unroll
-    for (int i = 0; i < (SUB * 16) / kThreads; ++i) {
-      const int idx = tid + i * kThreads;
-      const int row = idx >> 4, u = idx & 15;
-      const int key = base + row;
-      const bool ok = key < n_here;
-      const int slot = ok ? slot_of(tok0 + key) : 0;
-      cp_async16(sV + row * kVRow + ((u ^ (row & 7)) << 4), vbase + (seq0 + slot) * vrow_stride + u * 8,
-                 ok ? 16u : 0u);
+      for (int pp = 0; pp < kKRow / 128; ++pp) cp_async16(sk + pp * 128, kg + pp * 64, sz);
+#pragma unroll
+      for (int pp = 0; pp < kVRow / 128; ++pp) cp_async16(sv + pp * 128, vg + pp * 64, sz);
     }
   };
 
