@@ -76,16 +76,24 @@ __global__ void __launch_bounds__(kDecThreads, 4) select_score_kernel(const Sele
   for (int i = tid; i < 256; i += kDecThreads) s_h[i] = 0;   // first use is after a barrier
   const __nv_bfloat16* kbase = p.k + (static_cast<long long>(b) * p.seq_stride) * p.Hkv * kDQK + g * kDQK;
   const long long krow_stride = static_cast<long long>(p.Hkv) * kDQK;
+  // Thread t serves rows 16 i + t / 8 of the subtile and, in each, the 16-byte units 8 p + t % 8:
+  // every warp instruction reads 128 contiguous bytes from each of 4 rows, and a row is resolved
+  // once for all of its units.
   auto load_sub = [&](int st, int stage) {
     const uint32_t sK = s_base + stage * (kDecSub * kKRow);
+    const int lr = tid >> 3, lu = tid & 7;
 #pragma unroll
-    for (int i = 0; i < (kDecSub * 24) / kDecThreads; ++i) {
-      const int idx = tid + i * kDecThreads;
-      const int row = idx / 24, u = idx - row * 24;
+    for (int i = 0; i < kDecSub / (kDecThreads / 8); ++i) {
+      const int row = (kDecThreads / 8) * i + lr;
       const int key = st * kDecSub + row;
       const bool ok = key < n_here;
       const int t = ok ? k_begin + key : 0;
-      cp_async16(sK + row * kKRow + ((u ^ (row & 7)) << 4), kbase + t * krow_stride + u * 8, ok ? 16u : 0u);
+      const uint32_t sz = ok ? 16u : 0u;
+      const __nv_bfloat16* kg = kbase + t * krow_stride + lu * 8;
+      // unit 8 p + lu lands at unit 8 p + (lu ^ (row & 7)) (the XOR keeps the low 3 bits)
+      const uint32_t sk = sK + row * kKRow + static_cast<uint32_t>((lu ^ (row & 7)) << 4);
+#pragma unroll
+      for (int pp = 0; pp < kKRow / 128; ++pp) cp_async16(sk + pp * 128, kg + pp * 64, sz);
     }
   };
   const int nsub = (n_here + kDecSub - 1) / kDecSub;
