@@ -33,7 +33,8 @@ namespace mimo {
 
 // Optional per-tile timestamps (debug builds with -DMIMO_TRACE; compiled out otherwise):
 // events 0/1 S issued (group A/B), 2/3 PV issued, 4/5 S seen by the softmax group, 6/7 P
-// written, 9 K tile rotated, 10/11 S issue started, 12/13 PV issue started.
+// written, 9 K tile rotated, 10/11 S issue started, 12/13 PV issue started, 14/15 row max
+// done, 18/19 first half of P written.
 #ifdef MIMO_TRACE
 #define GA_TRACE(tile, ev)                                                             \
   do {                                                                                 \
@@ -476,6 +477,7 @@ __global__ void __launch_bounds__(kGaThreads, 1)
             }
           }
         }
+        if (q4 == 0 && lane == 0) GA_TRACE(gt, 14 + grp);
         const float tmax = fmaxf(mx0, mx1) * p.scale_log2;
         // Reference update: the first tile of a row moves it to the tile max (the dominant P
         // is then exactly 1); later tiles move it only when their max is 2^8 above it, so
@@ -533,6 +535,7 @@ __global__ void __launch_bounds__(kGaThreads, 1)
               }
               tmem_st8(trow + (c >> 1) + 8 * q, pk);
             }
+            if (c == 0 && q4 == 0 && lane == 0) GA_TRACE(gt, 18 + grp);
           }
         };
         if (full)
