@@ -41,6 +41,7 @@ struct DecodeMqParams {
   int B, T, Hq, Hkv, cap, mode, window, chunk, nchunks, direct;
   float scale_log2;
   unsigned* err;
+  unsigned long long* trace;  // debug timestamps (builds with -DMIMO_TRACE only), else null
 };
 
 // Key range [klo, L) of unit (b, .): the union of the draft tokens' key sets.

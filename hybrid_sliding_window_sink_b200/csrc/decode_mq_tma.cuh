@@ -13,9 +13,9 @@
 //    64-dim V slabs, 128-byte swizzle: the K-major B operand of S and the MN-major B operand of
 //    PV), four subtiles in flight.
 //  * warp 5, the MMA issuer (and TMEM allocator): S_j = Q K_j^T (N = 64, K = 192) into one of
-//    two TMEM buffers, then O += P_j V_j (N = 128, K = 64) with P from shared memory and O in
-//    TMEM; S_{j+1} is issued before PV_j, so the tensor core computes the next scores while the
-//    warps take this subtile's softmax.
+//    two TMEM buffers, O += P_j V_j (N = 128, K = 64) with P from shared memory and O in TMEM.
+//    Once P_j is written it issues PV_j and S_{j+2} together (one fence, one commit), so the
+//    tensor core computes those while the warps take the softmax of subtile j + 1.
 //  * warps 0-3, the softmax: with M = 64 row r of an accumulator sits in TMEM lane
 //    32 (r / 16) + r % 16, so warp w owns rows 16 w .. 16 w + 15 and reads them with
 //    tcgen05.ld.16x256b (rows gq and gq + 8 of each thread, columns 2 tq, 2 tq + 1 of every 8).
@@ -34,6 +34,21 @@
 #include "decode_mq.cuh"
 
 namespace mimo {
+
+// Optional per-subtile timestamps (debug builds with -DMIMO_TRACE; compiled out otherwise), for
+// the first chunk of KV head 0 of sequences 0-7: events 0 S issued, 1 PV issued, 2 S seen by the
+// softmax, 3 P written, 4 K/V subtile loads issued.
+#ifdef MIMO_TRACE
+#define MT_TRACE(sub, ev)                                                                       \
+  do {                                                                                          \
+    if (p.trace && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z < 8 && (sub) < 256)         \
+      p.trace[(static_cast<size_t>(blockIdx.z) * 256 + (sub)) * 32 + (ev)] = clock64();         \
+  } while (0)
+#else
+#define MT_TRACE(sub, ev) \
+  do {                    \
+  } while (0)
+#endif
 
 constexpr int kMtThreads = 192;
 constexpr int kMtKeys = 64;                                   // keys per subtile
@@ -54,10 +69,10 @@ constexpr uint32_t kMtIdescPV = idesc_bf16(64, kDV, 0, 1);
 enum : int {
   kMtKVFull = 0,                      // [4] K and V of a subtile landed
   kMtKVEmpty = kMtKVFull + kMtStages, // [4] PV of that subtile done: the stage is free
-  kMtSFull = kMtKVEmpty + kMtStages,  // [2] S written to a TMEM buffer
-  kMtPReady = kMtSFull + 2,           // [2] P written (128 arrivals): S buffer read, P buffer full
-  kMtPVDone = kMtPReady + 2,          // [2] PV read that P buffer and updated O
-  kMtFinal = kMtPVDone + 2,
+  kMtDone = kMtKVEmpty + kMtStages,   // [4] batch j (PV_j, S_{j+2}) done, in barrier j % 4
+  kMtInit = kMtDone + kMtStages,      // S_0 and S_1 done
+  kMtPReady = kMtInit + 1,            // [2] P written (128 arrivals): S buffer read, P buffer full
+  kMtFinal = kMtPReady + 2,
   kMtNumBars = kMtFinal + 1
 };
 
@@ -164,6 +179,7 @@ __global__ void __launch_bounds__(kMtThreads, 1)
           tma_load_4d(sK + s * kMtKBytes + cc * kMtSlab, &tmK, bar(kMtKVFull + s), 64 * cc, g, key0, b);
         for (int cc = 0; cc < 2; ++cc)
           tma_load_4d(sV + s * kMtVBytes + cc * kMtSlab, &tmV, bar(kMtKVFull + s), 64 * cc, g, key0, b);
+        MT_TRACE(j, 4);
       }
       if (!ok)   // let every issued copy land before the CTA can exit
         for (int t = j - kMtStages < 0 ? 0 : j - kMtStages; t < j; ++t)
@@ -171,55 +187,54 @@ __global__ void __launch_bounds__(kMtThreads, 1)
     }
   } else if (warp == 5) {
     // ------------------------------------------------------------ MMA issuer
+    // Batches: S_0 and S_1 first; then, once P_j is written, batch j = PV_j and S_{j+2} (which
+    // overwrites the S buffer P_j was taken from) under one fence. A tcgen05 fence or commit
+    // between two MMAs makes the issuing thread wait for the MMAs in flight, so a batch holds
+    // one commit besides its last: after PV_j, which frees the K/V stage for the producer.
     if (lane == 0) {
-      int ns = 0, npv = 0;
       bool ok = true;
-      uint32_t idle = 0;
-      unsigned long long t_prog = globaltimer_ns();
-      while (npv < nsub && ok) {
-        bool prog = false;
-        // S_ns: its K landed and its TMEM buffer read by the softmax of subtile ns - 2
-        if (ns < nsub && mbar_test(bar(kMtKVFull + ns % kMtStages), (ns / kMtStages) & 1) &&
-            (ns < 2 || mbar_test(bar(kMtPReady + (ns & 1)), ((ns >> 1) - 1) & 1))) {
-          tc_fence_after();
-          const uint32_t kb = sK + (ns % kMtStages) * kMtKBytes;
+      auto wait = [&](int i, int par) {
+        if (ok && !mbar_wait(bar(i), static_cast<uint32_t>(par & 1), s_abort, err)) ok = false;
+      };
+      auto issue_s = [&](int j) {
+        const uint32_t kb = sK + (j % kMtStages) * kMtKBytes;
 #pragma unroll
-          for (int kk = 0; kk < 12; ++kk) {
-            const uint64_t a = smem_desc(sQ + (kk >> 2) * kMtSlab + (kk & 3) * 32, 16, 1024);
-            const uint64_t bd = smem_desc(kb + (kk >> 2) * kMtSlab + (kk & 3) * 32, 16, 1024);
-            umma_ss(tmem + (ns & 1) * kMtKeys, a, bd, kMtIdescS, kk > 0 ? 1u : 0u);
-          }
-          umma_commit(bar(kMtSFull + (ns & 1)));
-          ++ns;
-          prog = true;
+        for (int kk = 0; kk < 12; ++kk) {
+          const uint64_t a = smem_desc(sQ + (kk >> 2) * kMtSlab + (kk & 3) * 32, 16, 1024);
+          const uint64_t bd = smem_desc(kb + (kk >> 2) * kMtSlab + (kk & 3) * 32, 16, 1024);
+          umma_ss(tmem + (j & 1) * kMtKeys, a, bd, kMtIdescS, kk > 0 ? 1u : 0u);
         }
-        // PV_npv: its P written
-        if (npv < ns && mbar_test(bar(kMtPReady + (npv & 1)), (npv >> 1) & 1)) {
-          tc_fence_after();
-          const uint32_t pb = sP + (npv & 1) * kMtSlab, vb = sV + (npv % kMtStages) * kMtVBytes;
+        MT_TRACE(j, 0);
+      };
+      auto issue_pv = [&](int j) {
+        const uint32_t pb = sP + (j & 1) * kMtSlab, vb = sV + (j % kMtStages) * kMtVBytes;
 #pragma unroll
-          for (int s2 = 0; s2 < kMtKeys / 16; ++s2) {
-            const uint64_t a = smem_desc(pb + s2 * 32, 16, 1024);
-            const uint64_t bd = smem_desc(vb + s2 * 2048, kMtSlab, 1024);
-            umma_ss(tmem + 128, a, bd, kMtIdescPV, (npv > 0 || s2 > 0) ? 1u : 0u);
-          }
-          umma_commit(bar(kMtPVDone + (npv & 1)));
-          umma_commit(bar(kMtKVEmpty + npv % kMtStages));
-          ++npv;
-          prog = true;
+        for (int s2 = 0; s2 < kMtKeys / 16; ++s2) {
+          const uint64_t a = smem_desc(pb + s2 * 32, 16, 1024);
+          const uint64_t bd = smem_desc(vb + s2 * 2048, kMtSlab, 1024);
+          umma_ss(tmem + 128, a, bd, kMtIdescPV, (j > 0 || s2 > 0) ? 1u : 0u);
         }
-        if (prog) {
-          idle = 0;
-        } else if ((++idle & 1023u) == 0) {
-          if (idle == 1024u) t_prog = globaltimer_ns();
-          if (*s_abort) {
-            ok = false;
-          } else if (globaltimer_ns() - t_prog > kWaitLimitNs) {
-            *s_abort = 1;
-            atomicOr(err, kErrWaitTimeout);
-            ok = false;
-          }
+        MT_TRACE(j, 1);
+      };
+      if (nsub > 0) {
+        wait(kMtKVFull, 0);
+        if (nsub > 1) wait(kMtKVFull + 1, 0);
+        if (ok) {
+          tc_fence_after();
+          issue_s(0);
+          if (nsub > 1) issue_s(1);
+          umma_commit(bar(kMtInit));
         }
+      }
+      for (int j = 0; j < nsub && ok; ++j) {
+        wait(kMtPReady + (j & 1), j >> 1);
+        if (j + 2 < nsub) wait(kMtKVFull + (j + 2) % kMtStages, (j + 2) / kMtStages);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(j);
+        umma_commit(bar(kMtKVEmpty + j % kMtStages));   // the producer may refill the stage now
+        if (j + 2 < nsub) issue_s(j + 2);
+        umma_commit(bar(kMtDone + j % kMtStages));
       }
       umma_commit(bar(kMtFinal));
       mbar_wait_drain(bar(kMtFinal), 0, err);
@@ -240,7 +255,12 @@ __global__ void __launch_bounds__(kMtThreads, 1)
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
     bool ok = true;
     for (int j = 0; j < nsub; ++j) {
-      if (!wait_all(bar(kMtSFull + (j & 1)), (j >> 1) & 1)) { ok = false; break; }
+      // S_j: in the first batch for j < 2, else in batch j - 2 (which also freed P buffer j & 1)
+      if (!wait_all(bar(j < 2 ? kMtInit : kMtDone + (j - 2) % kMtStages), j < 2 ? 0u : ((j - 2) / kMtStages) & 1)) {
+        ok = false;
+        break;
+      }
+      if (warp == 0 && lane == 0) MT_TRACE(j, 2);
       tc_fence_after();
       uint32_t sr[32];
       tmem_ld_16x256b_x8(trow + (j & 1) * kMtKeys, sr);
@@ -282,7 +302,7 @@ __global__ void __launch_bounds__(kMtThreads, 1)
       if (mv1) { a1 = ex2(m1 - mx1); m1 = mx1; l1 *= a1; }
       if (j > 0 && __any_sync(0xffffffffu, mv0 || mv1)) {
         // O must hold the PV of subtile j - 1 first
-        if (!wait_all(bar(kMtPVDone + ((j - 1) & 1)), ((j - 1) >> 1) & 1)) { ok = false; break; }
+        if (!wait_all(bar(kMtDone + (j - 1) % kMtStages), ((j - 1) / kMtStages) & 1)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll 1
         for (int hh = 0; hh < 2; ++hh) {
@@ -301,8 +321,7 @@ __global__ void __launch_bounds__(kMtThreads, 1)
         tmem_wait_st();
       }
       const float ref0 = m0 == -INFINITY ? 0.f : m0, ref1 = m1 == -INFINITY ? 0.f : m1;
-      // the P buffer was last read by PV of subtile j - 2
-      if (j >= 2 && !wait_all(bar(kMtPVDone + (j & 1)), ((j - 2) >> 1) & 1)) { ok = false; break; }
+      // (the P buffer was last read by PV of subtile j - 2, in the batch waited for above)
       const uint32_t pb = sP + (j & 1) * kMtSlab;
       float sum0 = 0.f, sum1 = 0.f;
 #pragma unroll
@@ -333,13 +352,14 @@ __global__ void __launch_bounds__(kMtThreads, 1)
       }
       fence_proxy_async_smem();
       tc_fence_before();
+      if (warp == 0 && lane == 0) MT_TRACE(j, 3);
       mbar_arrive(bar(kMtPReady + (j & 1)));
     }
     if (ok) {
       // O after the last PV; rows past R are not written
       float o[16][4];
       if (nsub > 0) {
-        if (!wait_all(bar(kMtPVDone + ((nsub - 1) & 1)), ((nsub - 1) >> 1) & 1)) ok = false;
+        if (!wait_all(bar(kMtDone + (nsub - 1) % kMtStages), ((nsub - 1) / kMtStages) & 1)) ok = false;
         tc_fence_after();
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {

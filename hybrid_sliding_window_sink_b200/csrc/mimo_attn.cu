@@ -632,6 +632,9 @@ mimo_status launch_decode_mq_tma_g(const mimo::DecodeMqParams& prm, cudaStream_t
     return MIMO_ERR_CUDA;
   }
   dim3 grid(prm.nchunks, prm.Hkv, prm.B);
+#ifdef MIMO_TRACE
+  const_cast<mimo::DecodeMqParams&>(prm).trace = g_trace;
+#endif
   kern<<<grid, mimo::kMtThreads, mimo::kMtSmemBytes, st>>>(tk, tv, prm);
   if (cudaGetLastError() != cudaSuccess) return MIMO_ERR_CUDA;
   if (!prm.direct) {
