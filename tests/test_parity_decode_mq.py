@@ -42,6 +42,8 @@ def test_ring(cuda_device, B, T, hq, hkv, cap, lengths):
     (3, 4, 64, 4, 200, [4, 64, 200]),           # one chunk
     (1, 1, 64, 4, 2500, [2500]),
     (2, 3, 32, 4, 1500, [700, 1500]),           # 3 draft tokens x 8 heads
+    (2, 4, 64, 4, 200, [100, 130]),             # one chunk of two and of three 64-key subtiles
+    (2, 4, 64, 4, 1200, [612, 1200]),           # last chunk of two subtiles after full ones
 ])
 def test_linear(cuda_device, B, T, hq, hkv, cap, lengths):
     _check(B, T, hq, hkv, "linear", cap, lengths, 0, cuda_device, seed=700 + T + cap)
